@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the base + log recurrent-state decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--log-cap L] [--batch B]
+
+A step is one decode step of the whole batch over all layers of the workload (one
+library call per layer), with every slot advancing by one token; merges happen on
+each slot's own merge step inside the same call.  Inputs are seeded synthetic
+tensors resident in HBM before timing starts.  L2 (126 MB) is flushed by writing a
+256 MiB buffer before every timed step, outside the timed interval; each step is
+bracketed by CUDA events on the launching stream.
+
+Multi-GPU (torchrun, one process per GPU): the slots are independent, so each rank
+runs its own replica of the workload (weak scaling, no collective on the data
+path); the reported time is the max over ranks.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle of
+the eager recurrence on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "decode head-steps/s (batch x heads x layers)"
+UNIT = "head-steps/s"
+FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "step_kernel_traffic.txt")
+KERNEL_SRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc", "dl_kernels.cuh")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gla_rwkv6_diag")
+    ap.add_argument("--log-cap", type=int, default=None)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-eager", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def workload(a):
+    from recurrent_state_serving_b200 import synth
+    wl = synth.WORKLOADS[a.workload]
+    if a.log_cap:
+        wl = wl.with_(log_cap=a.log_cap)
+    if a.batch:
+        wl = wl.with_(batch=a.batch)
+    return wl
+
+
+def config_of(wl, n_gpus):
+    return {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}",
+            "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
+            "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
+            "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
+            "l2": "flushed: 256 MiB write before every timed step, outside the timed interval",
+            "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    return 6650.0, "fallback (6.65 TB/s)"
+
+
+def recorded_traffic(workload_key):
+    """Per-launch DRAM bytes of the step kernel from a committed ncu summary, or None
+    when the summary is missing or the kernel source changed since it was taken."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    kv = {}
+    for line in open(PROFILE_TRAFFIC):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    src_hash = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+    if kv.get("kernel_sha") != src_hash or kv.get("workload") != workload_key:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.windows = []
+        self.proc = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = ["-i", str(device_index)]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        inside = [r for (t, r) in self.rows if any(a - 0.05 <= t <= b + 0.05 for a, b in self.windows)]
+        rows = inside or [r for _, r in self.rows]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                smax.append(float(r[1]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_in_timed_windows": len(inside)}
+
+
+# ---------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------
+def run_gpu(a, wl, rank, world, dist):
+    import torch
+    from recurrent_state_serving_b200 import deltalog as dl
+    from recurrent_state_serving_b200 import synth, traffic
+    from recurrent_state_serving_b200.runner import DecodeRunner
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    L, K, W = wl.log_cap, a.steps, a.warmup
+    ndist = max(1, min(wl.steps, 256 // wl.n_layers))
+
+    def barrier_sync():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def reduce_max(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    host_inputs = [[synth.step_inputs(wl, t, l) for l in range(wl.n_layers)] for t in range(ndist)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+
+    def timed(runner, calls_for_step, n_steps, pre=None):
+        """calls_for_step(i) -> list of callables issued for step i (one per layer)."""
+        for i in range(W):
+            for c in calls_for_step(i):
+                c()
+        barrier_sync()
+        t0 = time.time()
+        evs = []
+        for i in range(n_steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for c in calls_for_step(W + i):
+                c()
+            e1.record()
+            evs.append((e0, e1))
+        barrier_sync()
+        sampler.mark(t0, time.time())
+        ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+        return ms
+
+    # ---- deferred (the product path) ----
+    r = DecodeRunner(wl, device=str(dev))
+    r.load_initial_state()
+    r.run_presteps()
+    dev_inputs = [[r.device_inputs(x) for x in per_layer] for per_layer in host_inputs]
+    outs = [torch.empty(wl.batch, wl.n_heads, wl.d_v, dtype=torch.float32, device=dev)
+            for _ in range(wl.n_layers)]
+    prepared = [[dl.PreparedStep("decode", r.pool, l, r.slots, x["q"], x["k"], x["v"], x["lam"],
+                                 x["beta"], outs[l], wl.lambda_const) for l, x in enumerate(per_layer)]
+                for per_layer in dev_inputs]
+
+    def check(st):
+        if st != 0:
+            raise dl.DeltaLogError(st, "dl_decode_step")
+
+    calls = lambda i: [(lambda p=p: check(p())) for p in prepared[i % ndist]]
+    ms = timed(r, calls, K)
+    assert r.errors() == 0, "device error bits set during the benchmark"
+    total_ms = sum(ms)
+    max_ms = reduce_max(total_ms)
+    units = wl.units_per_step * K * world
+    value = units / (max_ms / 1e3)
+
+    # algorithmic bytes of the timed launches: slot b enters timed step i with
+    # c = (offset_b + W + i) mod L live entries (auto-merge cycle of length L)
+    offs = synth.slot_offsets(wl)
+    bytes_total = 0.0
+    for i in range(K):
+        c = (offs + W + i) % L
+        per_slot = [traffic.deferred_head_step(wl, int(cb), merge=(cb == L - 1)) for cb in c]
+        bytes_total += sum(per_slot) * wl.n_heads * wl.n_layers
+    launches = K * wl.n_layers
+    achieved_gbs = bytes_total / (total_ms / 1e3) / 1e9
+    peak, peak_src = measured_peaks()
+    key = config_of(wl, world)["workload"]
+    dram = recorded_traffic(key)
+    roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved_gbs / peak, 4), "peak_source": peak_src,
+            "traffic": dram, "algorithmic_bytes_per_launch": round(bytes_total / launches),
+            "kernel": "dl::step_kernel", "launches_timed": launches,
+            "avg_launch_us": round(total_ms * 1e3 / launches, 3),
+            "frac_of_8tbs_spec": round(achieved_gbs / 8000.0, 4)}
+
+    result = {"value": value, "ms_per_step": max_ms / K, "roofline": roof, "gpu_launches": launches}
+
+    # ---- eager comparison (same workload, full read-modify-write each step) ----
+    if not a.no_eager:
+        re_ = DecodeRunner(wl, device=str(dev), mode="eager")
+        re_.load_initial_state()
+        prep_e = [[dl.PreparedStep("eager", re_.pool, l, re_.slots, x["q"], x["k"], x["v"], x["lam"],
+                                   x["beta"], outs[l], wl.lambda_const) for l, x in enumerate(per_layer)]
+                  for per_layer in dev_inputs]
+        calls_e = lambda i: [(lambda p=p: check(p())) for p in prep_e[i % ndist]]
+        ms_e = timed(re_, calls_e, K)
+        assert re_.errors() == 0
+        tot_e = reduce_max(sum(ms_e))
+        eb = traffic.eager_head_step(wl) * wl.units_per_step * K
+        result["eager"] = {"value": wl.units_per_step * K * world / (tot_e / 1e3),
+                           "ms_per_step": tot_e / K,
+                           "algorithmic_bytes_per_step": round(eb / K),
+                           "achieved_gbs": round(eb / (sum(ms_e) / 1e3) / 1e9, 1)}
+        result["deferred_bytes_per_step"] = round(bytes_total / K)
+        del re_, prep_e
+        torch.cuda.empty_cache()
+
+    # ---- end to end through the public API with host buffers ----
+    if not a.no_e2e:
+        pin = lambda t: None if t is None else t.cpu().pin_memory()
+        host_dev = [[{k: pin(v) for k, v in x.items()} for x in per_layer] for per_layer in dev_inputs]
+        stage = [{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
+                 for x in dev_inputs[0]]
+        out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        prep_2 = [dl.PreparedStep("decode", r.pool, l, r.slots, s["q"], s["k"], s["v"], s["lam"],
+                                  s["beta"], outs[l], wl.lambda_const) for l, s in enumerate(stage)]
+        h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_calls(i):
+            src = host_dev[i % ndist]
+            cs = []
+            for l in range(wl.n_layers):
+                def one(l=l, src=src):
+                    for k, v in src[l].items():
+                        if v is not None:
+                            stage[l][k].copy_(v, non_blocking=True)
+                    check(prep_2[l]())
+                    out_host[l].copy_(outs[l], non_blocking=True)
+                cs.append(one)
+            return cs
+
+        ms_2 = timed(r, e2e_calls, K)
+        assert r.errors() == 0
+        tot_2 = reduce_max(sum(ms_2))
+        result["e2e"] = {"value": wl.units_per_step * K * world / (tot_2 / 1e3), "unit": UNIT,
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                         "ms_per_step": tot_2 / K,
+                         "path": "pinned host inputs -> H2D copy -> dl_decode_step per layer -> D2H of o_t, all inside the events"}
+    result["clocks"] = sampler.stop()
+    return result
+
+
+# ---------------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------------
+def oracle_sample_rate(wl, target_s=10.0):
+    """fp64 eager oracle on the host cores over a bounded sample of the workload's
+    heads (layer 0); returns (head-steps/s, threads, description)."""
+    import oracle
+    from recurrent_state_serving_b200 import synth
+    threads = os.cpu_count() or 1
+    x = synth.step_inputs(wl, 0, 0)
+    S0 = synth.initial_state(wl.with_(batch=min(wl.batch, 64)), 0).astype(np.float64)
+    rows = np.arange(S0.shape[0])
+
+    def run(T):
+        seq = [synth.select_rows(wl, synth.step_inputs(wl, t, 0), rows) for t in range(T)]
+        f = lambda k, t: synth.input_to_f64(seq[t][k], wl.in_dtype)
+        Q = np.stack([f("q", t) for t in range(T)])
+        Kk = np.stack([f("k", t) for t in range(T)])
+        V = np.stack([f("v", t) for t in range(T)])
+        LAM = None
+        if wl.decay != "none":
+            LAM = seq[0]["lam"].astype(np.float64) if wl.lambda_const else np.stack(
+                [seq[t]["lam"].astype(np.float64) for t in range(T)])
+        BETA = np.stack([seq[t]["beta"].astype(np.float64) for t in range(T)]) if wl.update == "delta" else None
+        t0 = time.perf_counter()
+        oracle.eager_rollout(S0, Q, Kk, V, LAM, BETA, decay=wl.decay, update=wl.update,
+                             lambda_const=wl.lambda_const, threads=threads)
+        return time.perf_counter() - t0
+
+    dt = run(2)
+    heads = S0.shape[0] * wl.n_heads
+    per_step = dt / 2
+    T = int(max(2, min(512, target_s / max(per_step, 1e-6))))
+    dt = run(T)
+    rate = heads * T / dt
+    desc = (f"{heads} heads ({S0.shape[0]} slots x {wl.n_heads} heads, layer 0) x {T} steps of "
+            f"{wl.name}, fp64 eager oracle, {dt:.1f} s")
+    return rate, threads, desc
+
+
+def run_reference(a, wl):
+    """Reference arm: the oracle, one bounded sample of the workload per step."""
+    import oracle
+    from recurrent_state_serving_b200 import synth
+    threads = os.cpu_count() or 1
+    budget_s = 90.0
+    rows_all = np.arange(wl.batch)
+    probe, _, _ = oracle_sample_rate(wl.with_(batch=min(wl.batch, 8)), target_s=1.0)
+    per_step_heads = max(wl.n_heads, min(wl.units_per_step,
+                                         int(probe * budget_s / max(1, a.steps + a.warmup))))
+    n_rows = max(1, min(wl.batch, per_step_heads // wl.n_heads))
+    rows = rows_all[:n_rows]
+    S = synth.initial_state(wl, 0)[rows].astype(np.float64)
+    x = synth.step_inputs(wl, 0, 0)
+    xs = synth.select_rows(wl, x, rows)
+    f = lambda k: synth.input_to_f64(xs[k], wl.in_dtype)[None]
+    Q, Kk, V = f("q"), f("k"), f("v")
+    LAM = None
+    if wl.decay != "none":
+        LAM = xs["lam"].astype(np.float64) if wl.lambda_const else xs["lam"].astype(np.float64)[None]
+    BETA = xs["beta"].astype(np.float64)[None] if wl.update == "delta" else None
+    times = []
+    for i in range(a.warmup + a.steps):
+        t0 = time.perf_counter()
+        _, Sck = oracle.eager_rollout(S, Q, Kk, V, LAM, BETA, decay=wl.decay, update=wl.update,
+                                      lambda_const=wl.lambda_const, ckpts=[1], threads=threads)
+        S = Sck[0]
+        if i >= a.warmup:
+            times.append(time.perf_counter() - t0)
+    units = n_rows * wl.n_heads
+    value = units * a.steps / sum(times)
+    sample = (f"{units} of {wl.units_per_step} head-steps per step ({n_rows} slots x {wl.n_heads} heads, "
+              f"layer 0), fp64 eager oracle advanced one token per step")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    a = parse()
+    sys.path.insert(0, ROOT)
+    wl = workload(a)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(a, wl)), flush=True)
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    else:
+        torch.cuda.set_device(0)
+
+    res = run_gpu(a, wl, rank, world, dist)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; bf16 q/k/v, fp32 lambda/beta, fp32 state and log)",
+            "config": config_of(wl, world), "roofline": res["roofline"],
+            "gpu_launches": res["gpu_launches"],
+            "hbm_tbs": res["roofline"]["achieved"] / 1e3}
+    for k in ("eager", "deferred_bytes_per_step", "e2e", "clocks"):
+        if k in res:
+            line[k] = res[k]
+    if world == 1 and not a.no_cpu:
+        rate, cores, desc = oracle_sample_rate(wl)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

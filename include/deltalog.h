@@ -1,0 +1,206 @@
+/*
+ * deltalog.h -- C ABI of a B200 (sm_100a) library for the batched recurrent-state
+ * decode step of linear-attention models, executed base + log ("DeltaLog").
+ *
+ * Passages this interface follows (DeltaLog: Deferred Materialization of
+ * Recurrent States for Linear Attention Decoding, Lin, Sun, Sun):
+ *  - Background, Eq. 3 (the common decode form): per slot, layer and head,
+ *        S_t = Diag(exp(lambda_t)) S_{t-1} + a_t b_t^T,   o_t = S_t^T q_t,
+ *    with a_t = k_t; b_t = v_t for additive operators (linear attention, RetNet,
+ *    GLA, RWKV6) and b_t = beta_t (v_t - Shat^T k_t) for delta-rule operators
+ *    (DeltaNet, GDN, KDA), Shat = Diag(exp(lambda_t)) S_{t-1} by default.
+ *    Scalar decay shares one lambda over all d_k coordinates; diagonal decay
+ *    uses a per-key vector.
+ *  - Section 3 (append-merge cycle, Algorithm 1): append steps record the
+ *    compact factors in a bounded log and leave the dense base untouched; every
+ *    merge interval the log is folded into the base and cleared.
+ *  - Section 3 (physical state): dense fp32 base state, cumulative log-decay,
+ *    key/value log buffers, one log-decay snapshot per entry, live-log length.
+ *  - Section 3 (traffic model, logical state): the base plus the log represents
+ *        S = D(lbar) Sbar + sum_{i<live} D(lbar - Lambda_i) a_i b_i^T,
+ *    D(x) = Diag(exp(x)), at every step.
+ *  - Section 3.3 (GPU execution): value-tiled work units over (slot, head,
+ *    value tile); key-side replay coefficients q^T a_i and k^T a_i with the
+ *    row rescaling D(lbar - Lambda_i); a single owner commits the shared log
+ *    metadata; Merge rewrites each dense fp32 tile once.
+ *  - Section 4 (serving integration): prefill initialises the base; a fresh or
+ *    reused slot starts with an empty log.
+ *
+ * Memory.  The library allocates no device memory.  Every buffer below is
+ * caller-owned device memory (for example torch tensors) and must stay alive
+ * while a pool that names it is in use.  All float buffers are fp32, row-major,
+ * 16-byte aligned.
+ *
+ * Streams.  Every call is asynchronous on the given cudaStream_t (passed as
+ * void*, NULL = legacy default stream) except dl_read_error, which
+ * synchronises that stream.  Calls on the same (pool, layer) must be ordered
+ * on one stream; different layers may run concurrently.
+ *
+ * Errors.  Argument problems found on the host are returned as a dl_status
+ * before anything is launched.  Problems only the device can see (a slot id out
+ * of range, a full log, a corrupt log length, an eager step on a slot with a
+ * live log) set a bit in the pool's sticky device error word and the affected
+ * work item is skipped; nothing traps.  Read the word with dl_read_error.
+ */
+#ifndef DELTALOG_H
+#define DELTALOG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DL_OK = 0,
+    DL_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, misaligned buffer, bad layer */
+    DL_ERR_SHAPE = 2,        /* dimension outside the supported set               */
+    DL_ERR_DTYPE = 3,        /* input dtype not supported                         */
+    DL_ERR_UNSUPPORTED = 4,  /* operation needs a log but the pool has none       */
+    DL_ERR_CUDA = 5,         /* a CUDA runtime call or a launch failed            */
+    DL_ERR_DEVICE = 6        /* dl_read_error found device error bits set         */
+} dl_status;
+
+/* Decay granularity of lambda_t (Background, Table 1 as restated in the text). */
+typedef enum {
+    DL_DECAY_NONE = 0,    /* lambda = 0: linear attention, DeltaNet                 */
+    DL_DECAY_SCALAR = 1,  /* one value per head: RetNet, GDN                        */
+    DL_DECAY_DIAG = 2     /* one value per key coordinate: GLA, RWKV6, KDA          */
+} dl_decay;
+
+/* Update semantics: how b_t is formed (Background; Section 3.4 per operator). */
+typedef enum {
+    DL_UPDATE_ADD = 0,             /* b_t = v_t                                        */
+    DL_UPDATE_DELTA = 1,           /* b_t = beta_t (v_t - (Diag(exp lambda_t) S_{t-1})^T k_t) */
+    DL_UPDATE_DELTA_UNDECAYED = 2  /* b_t = beta_t (v_t - S_{t-1}^T k_t)               */
+} dl_update;
+
+typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
+
+/* Sticky device error bits (dl_read_error). */
+#define DL_EBIT_SLOT_RANGE 0x1  /* a slot id outside [0, n_slots)                    */
+#define DL_EBIT_LOG_FULL 0x2    /* append / decode without auto-merge on a full log   */
+#define DL_EBIT_LIVE_LOG 0x4    /* eager step on a slot whose log is not empty        */
+#define DL_EBIT_LOG_LEN 0x8     /* a stored live-log length outside [0, log_cap]     */
+
+/* Pool descriptor.  One pool covers n_slots request slots x n_layers
+ * linear-attention layers x n_heads value heads.
+ *
+ *  d_k in {16, 64, 128}; d_v a multiple of 16 in [16, 1024];
+ *  n_kheads divides n_heads (grouped value attention: v-head h reads the q/k of
+ *  k-head h / (n_heads / n_kheads));  1 <= log_cap <= 64.
+ *
+ *  state    [n_slots][n_layers][n_heads][d_k][d_v]  fp32 dense base state.  The
+ *           caller writes prefill states here, then resets the slot's log.
+ *  log      [n_slots][n_layers][n_heads][log_cap][2*d_k + d_v] fp32 ring.  Row i
+ *           holds entry i as [a_i (d_k) | b_i (d_v) | Lambda_i (d_k)]; scalar decay
+ *           uses Lambda_i[0] only; no decay leaves Lambda unused.  NULL makes an
+ *           eager-only pool (decode/append/merge/materialize then return
+ *           DL_ERR_UNSUPPORTED).
+ *  log_len  [n_slots][n_layers] int32 live-log length (entries 0..log_len-1 live).
+ *           Required with a log; optional (NULL) for an eager-only pool.
+ *  arrive   [n_slots][n_layers] int32 arrival counters used to commit log_len once
+ *           per call.  Must be zero when the pool is created; the library returns
+ *           them to zero at the end of every call.  Required with a log.
+ *  err_word [1] int32 sticky device error bits; zero it before first use.
+ *  tile_v   value-tile width B_V of a work unit (Section 3.3): 16 or 32 columns,
+ *           or 0 to choose per launch (32 unless that leaves fewer than two CTAs
+ *           per SM).  32 needs d_k >= 64 and d_v a multiple of 32.
+ *
+ * The cumulative log-decay lbar of a slot is not stored separately: it equals
+ * Lambda of the newest live entry (0 when the log is empty).
+ */
+typedef struct {
+    int32_t n_slots, n_layers, n_heads, n_kheads, d_k, d_v, log_cap;
+    dl_decay decay;
+    dl_update update;
+    int32_t tile_v;
+    float *state;
+    float *log;
+    int32_t *log_len;
+    int32_t *arrive;
+    int32_t *err_word;
+} dl_pool_desc;
+
+typedef struct dl_pool dl_pool;  /* opaque host-side handle */
+
+/* Inputs of one decode step of one layer for a batch of slots.
+ *  slots   device [batch] int32 slot ids, distinct within one call.  Row b of
+ *          every per-row tensor below belongs to slot slots[b].
+ *  q, k    device [batch][n_kheads][d_k] (in_dtype).  k is the key factor a_t.
+ *  v       device [batch][n_heads][d_v] (in_dtype).
+ *  lambda  fp32 log-decay (<= 0 for a decaying state):
+ *            lambda_per_head == 0: [batch][n_heads] (scalar) | [batch][n_heads][d_k] (diag)
+ *            lambda_per_head == 1: [n_heads] (scalar) | [n_heads][d_k] (diag), the
+ *                                  same for every row and step (RetNet)
+ *          NULL iff decay == DL_DECAY_NONE.
+ *  beta    device [batch][n_heads] fp32, delta rule only (else ignored).
+ *  out     device [batch][n_heads][d_v] fp32 output o_t.  Ignored by dl_append.
+ */
+typedef struct {
+    const int32_t *slots;
+    int32_t batch;
+    const void *q, *k, *v;
+    dl_dtype in_dtype;
+    const float *lambda;
+    int32_t lambda_per_head;
+    const float *beta;
+    float *out;
+} dl_step_args;
+
+/* Validate a descriptor and return a host handle recording it.  No device
+ * memory is allocated and no CUDA call is made. */
+dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool);
+dl_status dl_destroy_pool(dl_pool *pool);
+
+/* One decode step (Section 3.3, AppendDecode + Finalize, and the merge step of
+ * the append-merge cycle).  For each slot with c live entries:
+ *   c < log_cap - 1, or auto_merge == 0 and c < log_cap:
+ *       read o_t and, for the delta rule, the correction (Shat^T k_t) off the
+ *       read-only base plus the decayed log; append (k_t, b_t, lbar + lambda_t)
+ *       as entry c; live length c + 1.
+ *   auto_merge != 0 and c >= log_cap - 1 (the slot's merge step):
+ *       compute o_t the same way and write the fully materialised state S_t
+ *       (base, log and the token) to the base; live length 0.
+ *   auto_merge == 0 and c == log_cap: DL_EBIT_LOG_FULL, slot skipped.
+ * So with auto_merge the merge interval equals log_cap, and log_cap == 1 is
+ * the eager recurrence. */
+dl_status dl_decode_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
+                         int32_t auto_merge, void *stream);
+
+/* Append the step's factors only (no output, never merges).  For the delta rule
+ * the base is still read to form b_t.  A full log sets DL_EBIT_LOG_FULL. */
+dl_status dl_append(dl_pool *pool, int32_t layer, const dl_step_args *args, void *stream);
+
+/* Merge (Section 3.3): for each listed slot fold its live log into the base,
+ *   Sbar <- D(lbar) Sbar + sum_i D(lbar - Lambda_i) a_i b_i^T,
+ * one read-modify-write pass per value tile, then reset the live length. */
+dl_status dl_merge(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
+                   void *stream);
+
+/* Eager dense step (Background: one read-modify-write of the full state per
+ * token), the in-library comparison path.  Requires an empty log on every
+ * listed slot (else DL_EBIT_LIVE_LOG and the slot is skipped). */
+dl_status dl_eager_step(dl_pool *pool, int32_t layer, const dl_step_args *args, void *stream);
+
+/* Empty the logs of the listed slots on every layer (Section 4: a fresh or
+ * reused slot starts with an empty auxiliary representation; the base, which
+ * prefill writes, is left alone). */
+dl_status dl_reset_slots(dl_pool *pool, const int32_t *slots, int32_t batch, void *stream);
+
+/* Write the logical state of the listed slots (logical-state equation) to
+ * dense_out [batch][n_heads][d_k][d_v] fp32 (device); the pool is unchanged. */
+dl_status dl_materialize(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
+                         float *dense_out, void *stream);
+
+/* Synchronise `stream`, copy the device error word to *bits, and clear it when
+ * `clear` is non-zero.  Returns DL_ERR_DEVICE when any bit was set. */
+dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *stream);
+
+/* Static description of a status code. */
+const char *dl_status_string(dl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTALOG_H */

@@ -1,0 +1,226 @@
+// C ABI of the base + log recurrent-state decode library: argument validation,
+// launch-shape selection and error reporting.  The arithmetic lives in the
+// kernels (dl_kernels.cuh); nothing here computes on the host.
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include <cuda_runtime.h>
+
+#include "deltalog.h"
+#include "dl_internal.h"
+
+#define DL_API extern "C" __attribute__((visibility("default")))
+
+struct dl_pool {
+    dl_pool_desc d;
+};
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool dk_supported(int dk) { return dk == 16 || dk == 64 || dk == 128; }
+
+dl::KParams base_params(const dl_pool_desc &d, int layer) {
+    dl::KParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.state = d.state;
+    p.log = d.log;
+    p.log_len = d.log_len;
+    p.arrive = d.arrive;
+    p.err = d.err_word;
+    p.n_slots = d.n_slots;
+    p.n_layers = d.n_layers;
+    p.H = d.n_heads;
+    p.Hk = d.n_kheads;
+    p.dk = d.d_k;
+    p.dv = d.d_v;
+    p.L = d.log_cap;
+    p.E = 2 * d.d_k + d.d_v;
+    p.layer = layer;
+    return p;
+}
+
+void set_tiles(const dl_pool_desc &d, dl::KParams &p, int batch, int &bv) {
+    bv = d.tile_v ? d.tile_v : dl::pick_bv(p.dk, p.dv, (long long)batch * p.H * (p.dv / 32));
+    p.nv = p.dv / bv;
+}
+
+dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, bool need_out) {
+    if (!P || !a) return DL_ERR_INVALID_ARG;
+    const dl_pool_desc &d = P->d;
+    if (layer < 0 || layer >= d.n_layers) return DL_ERR_INVALID_ARG;
+    if (a->batch < 0) return DL_ERR_SHAPE;
+    if (a->batch == 0) return DL_OK;
+    if (a->batch > d.n_slots) return DL_ERR_SHAPE;
+    if (!a->slots || !a->q || !a->k || !a->v) return DL_ERR_INVALID_ARG;
+    if (a->in_dtype != DL_F32 && a->in_dtype != DL_BF16) return DL_ERR_DTYPE;
+    const uintptr_t esz = a->in_dtype == DL_F32 ? 4 : 2;
+    if (!aligned(a->q, esz) || !aligned(a->k, esz) || !aligned(a->v, esz)) return DL_ERR_INVALID_ARG;
+    if (d.decay != DL_DECAY_NONE && (!a->lambda || !aligned(a->lambda, 4))) return DL_ERR_INVALID_ARG;
+    if (a->lambda_per_head != 0 && a->lambda_per_head != 1) return DL_ERR_INVALID_ARG;
+    if (d.update != DL_UPDATE_ADD && (!a->beta || !aligned(a->beta, 4))) return DL_ERR_INVALID_ARG;
+    if (need_out && (!a->out || !aligned(a->out, 4))) return DL_ERR_INVALID_ARG;
+    if (!aligned(a->slots, 4)) return DL_ERR_INVALID_ARG;
+    return DL_OK;
+}
+
+dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_out,
+                   bool auto_merge, bool eager, void *stream) {
+    const dl_pool_desc &d = P->d;
+    dl::KParams p = base_params(d, layer);
+    p.slots = a->slots;
+    p.batch = a->batch;
+    p.q = a->q;
+    p.k = a->k;
+    p.v = a->v;
+    p.lam = d.decay == DL_DECAY_NONE ? nullptr : a->lambda;
+    p.lam_const = a->lambda_per_head;
+    p.beta = d.update == DL_UPDATE_ADD ? nullptr : a->beta;
+    p.out = want_out ? a->out : nullptr;
+    p.auto_merge = auto_merge ? 1 : 0;
+    p.eager = eager ? 1 : 0;
+    p.want_out = want_out ? 1 : 0;
+    p.undecayed = d.update == DL_UPDATE_DELTA_UNDECAYED ? 1 : 0;
+    int bv = 32;
+    set_tiles(d, p, a->batch, bv);
+    const cudaError_t e = dl::launch_step(p, bv, d.decay, d.update != DL_UPDATE_ADD,
+                                          a->in_dtype == DL_BF16,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DL_OK : DL_ERR_CUDA;
+}
+
+}  // namespace
+
+DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
+    if (!desc || !out_pool) return DL_ERR_INVALID_ARG;
+    *out_pool = nullptr;
+    const dl_pool_desc &d = *desc;
+    if (d.n_slots <= 0 || d.n_layers <= 0 || d.n_heads <= 0 || d.n_kheads <= 0)
+        return DL_ERR_SHAPE;
+    if (d.n_heads % d.n_kheads) return DL_ERR_SHAPE;
+    if (!dk_supported(d.d_k)) return DL_ERR_SHAPE;
+    if (d.d_v < 16 || d.d_v > 1024 || d.d_v % 16) return DL_ERR_SHAPE;
+    if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
+    if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32) return DL_ERR_SHAPE;
+    if (d.tile_v == 32 && (d.d_k < 64 || d.d_v % 32)) return DL_ERR_SHAPE;
+    if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
+    if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
+        return DL_ERR_INVALID_ARG;
+    if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
+        return DL_ERR_INVALID_ARG;
+    if (d.log && (!aligned(d.log, 16) || !d.log_len || !d.arrive)) return DL_ERR_INVALID_ARG;
+    if ((d.log_len && !aligned(d.log_len, 4)) || (d.arrive && !aligned(d.arrive, 4)))
+        return DL_ERR_INVALID_ARG;
+    // launch grids are one CTA per (row, head, 16-column tile)
+    if ((long long)d.n_slots * d.n_heads * (d.d_v / 16) > 0x7fffffffLL) return DL_ERR_SHAPE;
+    dl_pool *p = new (std::nothrow) dl_pool;
+    if (!p) return DL_ERR_INVALID_ARG;
+    p->d = d;
+    *out_pool = p;
+    return DL_OK;
+}
+
+DL_API dl_status dl_destroy_pool(dl_pool *pool) {
+    if (!pool) return DL_ERR_INVALID_ARG;
+    delete pool;
+    return DL_OK;
+}
+
+DL_API dl_status dl_decode_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
+                                int32_t auto_merge, void *stream) {
+    const dl_status s = check_step(pool, layer, args, true);
+    if (s != DL_OK || args->batch == 0) return s;
+    if (!pool->d.log) return DL_ERR_UNSUPPORTED;
+    return run_step(pool, layer, args, true, auto_merge != 0, false, stream);
+}
+
+DL_API dl_status dl_append(dl_pool *pool, int32_t layer, const dl_step_args *args, void *stream) {
+    const dl_status s = check_step(pool, layer, args, false);
+    if (s != DL_OK || args->batch == 0) return s;
+    if (!pool->d.log) return DL_ERR_UNSUPPORTED;
+    return run_step(pool, layer, args, false, false, false, stream);
+}
+
+DL_API dl_status dl_eager_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
+                               void *stream) {
+    const dl_status s = check_step(pool, layer, args, true);
+    if (s != DL_OK || args->batch == 0) return s;
+    return run_step(pool, layer, args, true, false, true, stream);
+}
+
+static dl_status merge_like(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
+                            float *dense_out, bool materialize, void *stream) {
+    if (!pool) return DL_ERR_INVALID_ARG;
+    const dl_pool_desc &d = pool->d;
+    if (layer < 0 || layer >= d.n_layers) return DL_ERR_INVALID_ARG;
+    if (batch < 0 || batch > d.n_slots) return DL_ERR_SHAPE;
+    if (batch == 0) return DL_OK;
+    if (!slots || !aligned(slots, 4)) return DL_ERR_INVALID_ARG;
+    if (materialize && (!dense_out || !aligned(dense_out, 16))) return DL_ERR_INVALID_ARG;
+    if (!d.log) return DL_ERR_UNSUPPORTED;
+    dl::KParams p = base_params(d, layer);
+    p.slots = slots;
+    p.batch = batch;
+    p.dense_out = dense_out;
+    int bv = 32;
+    set_tiles(d, p, batch, bv);
+    const cudaError_t e = dl::launch_merge(p, bv, d.decay, materialize,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DL_OK : DL_ERR_CUDA;
+}
+
+DL_API dl_status dl_merge(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
+                          void *stream) {
+    return merge_like(pool, layer, slots, batch, nullptr, false, stream);
+}
+
+DL_API dl_status dl_materialize(dl_pool *pool, int32_t layer, const int32_t *slots,
+                                int32_t batch, float *dense_out, void *stream) {
+    return merge_like(pool, layer, slots, batch, dense_out, true, stream);
+}
+
+DL_API dl_status dl_reset_slots(dl_pool *pool, const int32_t *slots, int32_t batch,
+                                void *stream) {
+    if (!pool) return DL_ERR_INVALID_ARG;
+    const dl_pool_desc &d = pool->d;
+    if (batch < 0 || batch > d.n_slots) return DL_ERR_SHAPE;
+    if (batch == 0) return DL_OK;
+    if (!slots || !aligned(slots, 4)) return DL_ERR_INVALID_ARG;
+    if (!d.log_len) return DL_OK;  // eager-only pool without a log: nothing to reset
+    const cudaError_t e = dl::launch_reset(slots, batch, d.n_slots, d.n_layers, d.log_len,
+                                           d.arrive, d.err_word,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DL_OK : DL_ERR_CUDA;
+}
+
+DL_API dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *stream) {
+    if (!pool || !bits) return DL_ERR_INVALID_ARG;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t host = 0;
+    if (cudaMemcpyAsync(&host, pool->d.err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+        return DL_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DL_ERR_CUDA;
+    if (clear && host) {
+        if (cudaMemsetAsync(pool->d.err_word, 0, sizeof(int32_t), st) != cudaSuccess)
+            return DL_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return DL_ERR_CUDA;
+    }
+    *bits = host;
+    return host ? DL_ERR_DEVICE : DL_OK;
+}
+
+DL_API const char *dl_status_string(dl_status status) {
+    switch (status) {
+    case DL_OK: return "ok";
+    case DL_ERR_INVALID_ARG: return "invalid argument";
+    case DL_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case DL_ERR_DTYPE: return "unsupported dtype";
+    case DL_ERR_UNSUPPORTED: return "operation not supported by this pool";
+    case DL_ERR_CUDA: return "CUDA error";
+    case DL_ERR_DEVICE: return "device error bits set";
+    }
+    return "unknown status";
+}

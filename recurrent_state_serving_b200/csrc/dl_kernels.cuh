@@ -1,0 +1,438 @@
+// sm_100a kernels of the base + log recurrent-state decode step.
+//
+// Work decomposition (DeltaLog paper, Section 3.3): one CTA per
+// (slot, head, value tile); the tile is the d_k x B_V slice of the head's dense
+// fp32 base state.  A head's N_V = d_v / B_V tiles are adjacent in blockIdx so the
+// key-side data they share (q, k, a_i, Lambda_i) is read from HBM once and hit in L2
+// by the others.
+//
+// Inside a CTA each thread owns RPT rows x 4 columns of the tile (one 128-bit
+// word per row).  A warp's load instruction covers 32/CQ whole rows of the tile
+// (128 B per row at B_V = 32), so every global access is a full, aligned line.
+// The tile is fetched into registers with cache-streaming 128-bit loads at the
+// top of the kernel, before any metadata is read, so the HBM stream is in flight
+// while the CTA computes its replay coefficients.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "dl_internal.h"
+
+namespace dl {
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <int DK, int BV> struct TileShape {
+    static constexpr int CQ = BV / 4;                     // 128-bit column words per row
+    static constexpr int NT = (DK * BV / 32) < 32 ? 32 : (DK * BV / 32);  // 8 words/thread
+    static constexpr int RG = NT / CQ;                    // row groups
+    static constexpr int RPT = DK / RG;                   // rows per thread
+    static constexpr int NW = NT / 32;                    // warps
+    static_assert(RPT * RG == DK, "tile rows must divide evenly");
+    static_assert(32 % CQ == 0 && NT % 32 == 0, "bad tile shape");
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ void fma4(float4 &acc, float a, const float4 &b) {
+    acc.x = fmaf(a, b.x, acc.x);
+    acc.y = fmaf(a, b.y, acc.y);
+    acc.z = fmaf(a, b.z, acc.z);
+    acc.w = fmaf(a, b.w, acc.w);
+}
+
+// Offsets (floats) inside the dynamic shared-memory block.
+struct DynLayout {
+    int cq, ck, b, A;
+    __device__ __forceinline__ DynLayout(int L, int bv) {
+        const int L4 = (L + 3) & ~3;
+        cq = 0;
+        ck = L4;
+        b = 2 * L4;
+        A = 2 * L4 + L * bv;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Decode / append / eager step.
+//
+// For the slot's c live entries and this step's token (paper, logical-state
+// equation with lbar_t = Lambda_{c-1} + lambda_t):
+//   qt = e^{lbar_t} (.) q,   kt = e^{lbar_t} (.) k   (e^{Lambda_{c-1}} for the
+//                                                     undecayed delta reading)
+//   cq_i = sum_r a_i[r] e^{lbar_t[r] - Lambda_i[r]} q[r]        (ReplayPrep)
+//   ck_i = the same with k                                      (delta rule)
+//   y_q = Sbar^T qt + sum_i cq_i b_i,  y_k = Sbar^T kt + sum_i ck_i b_i
+//   b_t = v (additive) | beta (v - y_k) (delta);  o_t = y_q + b_t (k . q)
+// then either append (k, b_t, lbar_t) as entry c, or, on the slot's merge step
+// (and always in eager mode), write
+//   S_t = e^{lbar_t} (.) Sbar + sum_i A'_i b_i^T + k b_t^T,  A'_i = a_i (.) e^{lbar_t - Lambda_i}.
+// ---------------------------------------------------------------------------
+template <int DK, int BV, int DECAY, bool DELTA, typename IT>
+__global__ void __launch_bounds__(TileShape<DK, BV>::NT)
+    step_kernel(const KParams p)
+{
+    using Sh = TileShape<DK, BV>;
+    constexpr int NT = Sh::NT, CQ = Sh::CQ, RG = Sh::RG, RPT = Sh::RPT, NW = Sh::NW;
+
+    __shared__ float s_q[DK], s_k[DK], s_qt[DK], s_kt[DK], s_ell[DK], s_ellp[DK], s_e[DK];
+    __shared__ float s_red[2][NW][BV];
+    __shared__ __align__(16) float s_bt[BV];
+    __shared__ float s_kq;
+    extern __shared__ __align__(16) float s_dyn[];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nv = p.nv;
+    const int j = blockIdx.x % nv;
+    const int h = (blockIdx.x / nv) % p.H;
+    const int bi = blockIdx.x / (nv * p.H);
+    const int dv = p.dv;
+
+    const int s = p.slots[bi];
+    if (s < 0 || s >= p.n_slots) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_SLOT_RANGE);
+        return;
+    }
+    const size_t sl = (size_t)s * p.n_layers + p.layer;
+    const size_t head = sl * p.H + h;
+    float *tile = p.state + head * (size_t)DK * dv + (size_t)j * BV;
+    const int quad = tid % CQ, rg = tid / CQ;
+
+    // 1. stream the base tile (read-only on append steps)
+    const bool need_base = p.want_out || DELTA || p.eager || p.auto_merge;
+    float4 Sr[RPT];
+    if (need_base) {
+#pragma unroll
+        for (int m = 0; m < RPT; ++m)
+            Sr[m] = __ldcs(reinterpret_cast<const float4 *>(tile + (size_t)(rg + m * RG) * dv) + quad);
+    }
+
+    // 2. live-log length and phase
+    int c = 0;
+    if (p.log_len) c = p.log_len[sl];
+    if (p.eager) {
+        if (c != 0) {
+            if (tid == 0) atomicOr(p.err, DL_EBIT_LIVE_LOG);
+            return;
+        }
+    } else if (c < 0 || c > p.L) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_LEN);
+        return;
+    }
+    const bool merge_now = p.eager || (p.auto_merge && c >= p.L - 1);
+    if (!merge_now && c >= p.L) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_FULL);
+        return;
+    }
+    float *ring = p.log ? p.log + head * (size_t)p.L * p.E : nullptr;
+    const DynLayout lay(p.L, BV);
+    float *s_cq = s_dyn + lay.cq, *s_ck = s_dyn + lay.ck, *s_b = s_dyn + lay.b, *s_A = s_dyn + lay.A;
+
+    // 3. token, cumulative log-decay, prescaled q and k
+    const int g = h / (p.H / p.Hk);
+    const IT *qrow = static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + g) * DK;
+    const IT *krow = static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + g) * DK;
+    const float *Lprev = (c > 0) ? ring + (size_t)(c - 1) * p.E + DK + dv : nullptr;
+    float lam_s = 0.f;
+    const float *lrow = nullptr;
+    if (DECAY == DL_DECAY_SCALAR) lam_s = p.lam_const ? p.lam[h] : p.lam[(size_t)bi * p.H + h];
+    if (DECAY == DL_DECAY_DIAG)
+        lrow = p.lam_const ? p.lam + (size_t)h * DK : p.lam + ((size_t)bi * p.H + h) * DK;
+    for (int r = tid; r < DK; r += NT) {
+        const float qv = to_f32(qrow[r]), kv = to_f32(krow[r]);
+        float lp = 0.f, lt = 0.f, et = 1.f, ek = 1.f;
+        if (DECAY == DL_DECAY_DIAG) {
+            lp = Lprev ? Lprev[r] : 0.f;
+            lt = lp + lrow[r];
+        } else if (DECAY == DL_DECAY_SCALAR) {
+            lp = Lprev ? Lprev[0] : 0.f;
+            lt = lp + lam_s;
+        }
+        if (DECAY != DL_DECAY_NONE) {
+            et = expf(lt);
+            ek = (DELTA && p.undecayed) ? expf(lp) : et;
+        }
+        s_q[r] = qv;
+        s_k[r] = kv;
+        s_ell[r] = lt;
+        s_ellp[r] = lp;
+        s_e[r] = et;
+        s_qt[r] = et * qv;
+        s_kt[r] = ek * kv;
+    }
+    __syncthreads();
+
+    // 4. ReplayPrep: key-side replay coefficients, one warp per log entry
+    for (int i = warp; i < c; i += NW) {
+        const float *ent = ring + (size_t)i * p.E;
+        float fs = 1.f, fk = 1.f;
+        if (DECAY == DL_DECAY_SCALAR) {
+            const float Li = ent[DK + dv];
+            fs = expf(s_ell[0] - Li);
+            fk = (DELTA && p.undecayed) ? expf(s_ellp[0] - Li) : fs;
+        }
+        float pq = 0.f, pk = 0.f;
+        for (int r4 = lane; r4 < DK / 4; r4 += 32) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(ent + 4 * r4);
+            float4 L4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (DECAY == DL_DECAY_DIAG) L4 = *reinterpret_cast<const float4 *>(ent + DK + dv + 4 * r4);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+            const float Lv[4] = {L4.x, L4.y, L4.z, L4.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int r = 4 * r4 + x;
+                float w, wk;
+                if (DECAY == DL_DECAY_DIAG) {
+                    w = av[x] * expf(s_ell[r] - Lv[x]);
+                    wk = (DELTA && p.undecayed) ? av[x] * expf(s_ellp[r] - Lv[x]) : w;
+                } else {
+                    w = av[x] * fs;
+                    wk = av[x] * fk;
+                }
+                pq = fmaf(w, s_q[r], pq);
+                if (DELTA) pk = fmaf(wk, s_k[r], pk);
+                if (merge_now) s_A[i * DK + r] = w;
+            }
+        }
+        pq = warp_sum(pq);
+        if (DELTA) pk = warp_sum(pk);
+        if (lane == 0) {
+            s_cq[i] = pq;
+            s_ck[i] = pk;
+        }
+    }
+    // value-side log shard of this tile
+    for (int idx = tid; idx < c * CQ; idx += NT) {
+        const int i = idx / CQ, x4 = idx % CQ;
+        reinterpret_cast<float4 *>(s_b + i * BV)[x4] =
+            *reinterpret_cast<const float4 *>(ring + (size_t)i * p.E + DK + (size_t)j * BV + 4 * x4);
+    }
+    if (p.want_out && warp == 0) {  // a_t . q_t for the new entry (no decay since insertion)
+        float x = 0.f;
+        for (int r = lane; r < DK; r += 32) x = fmaf(s_q[r], s_k[r], x);
+        x = warp_sum(x);
+        if (lane == 0) s_kq = x;
+    }
+    __syncthreads();
+
+    // 5. AppendDecode: base mat-vecs S^T qt and S^T kt over this tile
+    float yq[4] = {0.f, 0.f, 0.f, 0.f}, yk[4] = {0.f, 0.f, 0.f, 0.f};
+    if (need_base) {
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const int r = rg + m * RG;
+            const float a = s_qt[r];
+            yq[0] = fmaf(Sr[m].x, a, yq[0]);
+            yq[1] = fmaf(Sr[m].y, a, yq[1]);
+            yq[2] = fmaf(Sr[m].z, a, yq[2]);
+            yq[3] = fmaf(Sr[m].w, a, yq[3]);
+            if (DELTA) {
+                const float b = s_kt[r];
+                yk[0] = fmaf(Sr[m].x, b, yk[0]);
+                yk[1] = fmaf(Sr[m].y, b, yk[1]);
+                yk[2] = fmaf(Sr[m].z, b, yk[2]);
+                yk[3] = fmaf(Sr[m].w, b, yk[3]);
+            }
+        }
+#pragma unroll
+        for (int o = CQ; o < 32; o <<= 1) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                yq[x] += __shfl_xor_sync(0xffffffffu, yq[x], o);
+                if (DELTA) yk[x] += __shfl_xor_sync(0xffffffffu, yk[x], o);
+            }
+        }
+        if (lane < CQ) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                s_red[0][warp][4 * quad + x] = yq[x];
+                s_red[1][warp][4 * quad + x] = yk[x];
+            }
+        }
+    }
+    __syncthreads();
+
+    // 6. replay the value log, form b_t and o_t, append (or prepare the merge)
+    if (tid < BV) {
+        const int col = j * BV + tid;
+        float Yq = 0.f, Yk = 0.f;
+        if (need_base) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                Yq += s_red[0][w][tid];
+                Yk += s_red[1][w][tid];
+            }
+        }
+        for (int i = 0; i < c; ++i) {
+            const float b = s_b[i * BV + tid];
+            Yq = fmaf(b, s_cq[i], Yq);
+            if (DELTA) Yk = fmaf(b, s_ck[i], Yk);
+        }
+        const size_t row = (size_t)bi * p.H + h;
+        const float vv = to_f32(static_cast<const IT *>(p.v)[row * dv + col]);
+        const float bt = DELTA ? p.beta[row] * (vv - Yk) : vv;
+        if (p.want_out) p.out[row * dv + col] = fmaf(bt, s_kq, Yq);
+        if (!merge_now) ring[(size_t)c * p.E + DK + col] = bt;
+        s_bt[tid] = bt;
+    }
+    if (!merge_now && j == 0) {  // designated writer of the shared entry fields
+        float *ent = ring + (size_t)c * p.E;
+        for (int r = tid; r < DK; r += NT) {
+            ent[r] = s_k[r];
+            if (DECAY == DL_DECAY_DIAG) ent[DK + dv + r] = s_ell[r];
+        }
+        if (DECAY == DL_DECAY_SCALAR && tid == 0) ent[DK + dv] = s_ell[0];
+    }
+
+    // 7. merge step: write the materialised state back over the base tile
+    if (merge_now) {
+        __syncthreads();
+        const float4 btq = reinterpret_cast<const float4 *>(s_bt)[quad];
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const int r = rg + m * RG;
+            const float e = s_e[r];
+            Sr[m].x *= e;
+            Sr[m].y *= e;
+            Sr[m].z *= e;
+            Sr[m].w *= e;
+            fma4(Sr[m], s_k[r], btq);
+        }
+        for (int i = 0; i < c; ++i) {
+            const float4 b4 = reinterpret_cast<const float4 *>(s_b + i * BV)[quad];
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) fma4(Sr[m], s_A[i * DK + rg + m * RG], b4);
+        }
+#pragma unroll
+        for (int m = 0; m < RPT; ++m)
+            __stcs(reinterpret_cast<float4 *>(tile + (size_t)(rg + m * RG) * dv) + quad, Sr[m]);
+    }
+
+    // 8. Finalize: the last CTA of this (slot, layer) commits the live length
+    if (!p.eager) {
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const int total = p.H * nv;
+            const int old = atomicAdd(p.arrive + sl, 1);
+            if (old == total - 1) {
+                p.log_len[sl] = merge_now ? 0 : c + 1;
+                p.arrive[sl] = 0;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge / materialise: Sbar' = e^{lbar} (.) Sbar + sum_{i<c} A'_i b_i^T with
+// lbar = Lambda_{c-1}, A'_i = a_i (.) e^{lbar - Lambda_i}.  Merge writes Sbar' over
+// the base and resets the live length; materialise writes it to dense_out.
+// ---------------------------------------------------------------------------
+template <int DK, int BV, int DECAY>
+__global__ void __launch_bounds__(TileShape<DK, BV>::NT)
+    merge_kernel(const KParams p, const int materialize)
+{
+    using Sh = TileShape<DK, BV>;
+    constexpr int NT = Sh::NT, CQ = Sh::CQ, RG = Sh::RG, RPT = Sh::RPT;
+
+    __shared__ float s_e[DK];
+    extern __shared__ __align__(16) float s_dyn[];
+
+    const int tid = threadIdx.x;
+    const int nv = p.nv;
+    const int j = blockIdx.x % nv;
+    const int h = (blockIdx.x / nv) % p.H;
+    const int bi = blockIdx.x / (nv * p.H);
+    const int dv = p.dv;
+
+    const int s = p.slots[bi];
+    if (s < 0 || s >= p.n_slots) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_SLOT_RANGE);
+        return;
+    }
+    const size_t sl = (size_t)s * p.n_layers + p.layer;
+    const size_t head = sl * p.H + h;
+    float *tile = p.state + head * (size_t)DK * dv + (size_t)j * BV;
+    const int quad = tid % CQ, rg = tid / CQ;
+
+    const int c = p.log_len[sl];
+    if (c < 0 || c > p.L) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_LEN);
+        return;
+    }
+    if (!materialize && c == 0) return;  // nothing to fold; live length stays 0
+
+    float4 Sr[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m)
+        Sr[m] = __ldcs(reinterpret_cast<const float4 *>(tile + (size_t)(rg + m * RG) * dv) + quad);
+
+    const float *ring = p.log + head * (size_t)p.L * p.E;
+    const DynLayout lay(p.L, BV);
+    float *s_b = s_dyn + lay.b, *s_A = s_dyn + lay.A;
+    const float *Lbar = (c > 0) ? ring + (size_t)(c - 1) * p.E + DK + dv : nullptr;
+
+    for (int r = tid; r < DK; r += NT) {
+        float e = 1.f;
+        if (DECAY == DL_DECAY_DIAG && Lbar) e = expf(Lbar[r]);
+        if (DECAY == DL_DECAY_SCALAR && Lbar) e = expf(Lbar[0]);
+        s_e[r] = e;
+    }
+    for (int idx = tid; idx < c * DK; idx += NT) {
+        const int i = idx / DK, r = idx % DK;
+        const float *ent = ring + (size_t)i * p.E;
+        float w = ent[r];
+        if (DECAY == DL_DECAY_DIAG) w *= expf(Lbar[r] - ent[DK + dv + r]);
+        if (DECAY == DL_DECAY_SCALAR) w *= expf(Lbar[0] - ent[DK + dv]);
+        s_A[idx] = w;
+    }
+    for (int idx = tid; idx < c * CQ; idx += NT) {
+        const int i = idx / CQ, x4 = idx % CQ;
+        reinterpret_cast<float4 *>(s_b + i * BV)[x4] =
+            *reinterpret_cast<const float4 *>(ring + (size_t)i * p.E + DK + (size_t)j * BV + 4 * x4);
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const float e = s_e[rg + m * RG];
+        Sr[m].x *= e;
+        Sr[m].y *= e;
+        Sr[m].z *= e;
+        Sr[m].w *= e;
+    }
+    for (int i = 0; i < c; ++i) {
+        const float4 b4 = reinterpret_cast<const float4 *>(s_b + i * BV)[quad];
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) fma4(Sr[m], s_A[i * DK + rg + m * RG], b4);
+    }
+    float *dst = materialize
+                     ? p.dense_out + ((size_t)bi * p.H + h) * (size_t)DK * dv + (size_t)j * BV
+                     : tile;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m)
+        __stcs(reinterpret_cast<float4 *>(dst + (size_t)(rg + m * RG) * dv) + quad, Sr[m]);
+
+    if (!materialize) {
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const int old = atomicAdd(p.arrive + sl, 1);
+            if (old == p.H * nv - 1) {
+                p.log_len[sl] = 0;
+                p.arrive[sl] = 0;
+            }
+        }
+    }
+}
+
+}  // namespace dl

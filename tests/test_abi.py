@@ -1,0 +1,144 @@
+"""CPU tests of the C ABI: the library loads, exports what the header declares, and
+validates arguments on the host.  No call here reaches the GPU: every call either
+fails validation or is a no-op (batch == 0) before any CUDA runtime call."""
+import ctypes
+import subprocess
+
+import pytest
+
+from recurrent_state_serving_b200 import deltalog as dl
+
+EXPECTED = ["dl_append", "dl_create_pool", "dl_decode_step", "dl_destroy_pool",
+            "dl_eager_step", "dl_materialize", "dl_merge", "dl_read_error", "dl_reset_slots",
+            "dl_status_string"]
+
+
+def test_header_declares_the_boundary():
+    assert dl.header_functions() == EXPECTED
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(dl.LIB_PATH)
+    for name in dl.header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_only_the_abi_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", dl.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    text_syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert sorted(s for s in text_syms if s.startswith("dl_")) == EXPECTED
+    assert not [s for s in text_syms if "dl" in s and not s.startswith("dl_")]
+
+
+def _desc(**kw):
+    base = dict(n_slots=4, n_layers=2, n_heads=4, n_kheads=2, d_k=128, d_v=128, log_cap=8,
+                decay=2, update=1, tile_v=0, state=0x10000, log=0x20000, log_len=0x30000,
+                arrive=0x40000, err_word=0x50000)
+    base.update(kw)
+    return dl.dl_pool_desc(**base)
+
+
+def _create(desc):
+    h = ctypes.c_void_p()
+    st = dl.library().dl_create_pool(ctypes.byref(desc), ctypes.byref(h))
+    return st, h
+
+
+def test_create_pool_accepts_valid_descriptors():
+    for kw in ({}, dict(d_k=16, d_v=16, n_kheads=4), dict(d_k=64, d_v=80), dict(log_cap=1),
+               dict(log_cap=64), dict(log=None, log_len=None, arrive=None), dict(decay=0, update=0),
+               dict(tile_v=16), dict(tile_v=32), dict(d_k=64, d_v=96, tile_v=32)):
+        st, h = _create(_desc(**kw))
+        assert st == dl.DL_OK, (kw, dl.dl_status_string(st))
+        assert dl.library().dl_destroy_pool(h) == dl.DL_OK
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_slots=0), dl.DL_ERR_SHAPE),
+    (dict(n_heads=6, n_kheads=4), dl.DL_ERR_SHAPE),
+    (dict(d_k=32), dl.DL_ERR_SHAPE),
+    (dict(d_k=100), dl.DL_ERR_SHAPE),
+    (dict(d_v=40), dl.DL_ERR_SHAPE),
+    (dict(d_v=2048), dl.DL_ERR_SHAPE),
+    (dict(log_cap=0), dl.DL_ERR_SHAPE),
+    (dict(log_cap=65), dl.DL_ERR_SHAPE),
+    (dict(decay=3), dl.DL_ERR_INVALID_ARG),
+    (dict(update=-1), dl.DL_ERR_INVALID_ARG),
+    (dict(state=None), dl.DL_ERR_INVALID_ARG),
+    (dict(state=0x10004), dl.DL_ERR_INVALID_ARG),
+    (dict(err_word=None), dl.DL_ERR_INVALID_ARG),
+    (dict(log_len=None), dl.DL_ERR_INVALID_ARG),
+    (dict(arrive=None), dl.DL_ERR_INVALID_ARG),
+    (dict(log=0x20008), dl.DL_ERR_INVALID_ARG),
+    (dict(tile_v=8), dl.DL_ERR_SHAPE),
+    (dict(tile_v=32, d_k=16, d_v=32), dl.DL_ERR_SHAPE),
+    (dict(tile_v=32, d_v=80), dl.DL_ERR_SHAPE),
+])
+def test_create_pool_rejects(kw, status):
+    st, h = _create(_desc(**kw))
+    assert st == status
+    assert not h.value
+
+
+def test_step_argument_validation_without_gpu():
+    lib = dl.library()
+    st, h = _create(_desc())
+    assert st == dl.DL_OK
+    P = 0x60000
+    good = dict(slots=P, batch=2, q=P, k=P, v=P, in_dtype=1, lambda_=P, lambda_per_head=0,
+                beta=P, out=P)
+
+    def call(fn, **kw):
+        a = dict(good)
+        a.update(kw)
+        args = dl.dl_step_args(**a)
+        if fn == "dl_decode_step":
+            return lib.dl_decode_step(h, 0, ctypes.byref(args), 1, None)
+        return getattr(lib, fn)(h, 0, ctypes.byref(args), None)
+
+    for fn in ("dl_decode_step", "dl_append", "dl_eager_step"):
+        assert call(fn, batch=0) == dl.DL_OK                   # empty batch: no launch
+        assert call(fn, batch=-1) == dl.DL_ERR_SHAPE
+        assert call(fn, batch=5) == dl.DL_ERR_SHAPE            # more rows than slots
+        assert call(fn, slots=None) == dl.DL_ERR_INVALID_ARG
+        assert call(fn, q=None) == dl.DL_ERR_INVALID_ARG
+        assert call(fn, in_dtype=7) == dl.DL_ERR_DTYPE
+        assert call(fn, lambda_=None) == dl.DL_ERR_INVALID_ARG  # diag decay needs lambda
+        assert call(fn, beta=None) == dl.DL_ERR_INVALID_ARG     # delta rule needs beta
+        assert call(fn, lambda_per_head=2) == dl.DL_ERR_INVALID_ARG
+        assert call(fn, q=P + 1) == dl.DL_ERR_INVALID_ARG       # misaligned bf16
+    assert call("dl_decode_step", out=None) == dl.DL_ERR_INVALID_ARG
+    assert call("dl_eager_step", out=None) == dl.DL_ERR_INVALID_ARG
+    a = dl.dl_step_args(**good)
+    assert lib.dl_decode_step(h, 2, ctypes.byref(a), 1, None) == dl.DL_ERR_INVALID_ARG  # layer
+    assert lib.dl_decode_step(h, -1, ctypes.byref(a), 1, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_decode_step(None, 0, ctypes.byref(a), 1, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_merge(h, 0, P, 0, None) == dl.DL_OK
+    assert lib.dl_merge(h, 0, None, 1, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_merge(h, 3, P, 1, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_materialize(h, 0, P, 1, None, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_reset_slots(h, P, 0, None) == dl.DL_OK
+    assert lib.dl_reset_slots(h, P, 9, None) == dl.DL_ERR_SHAPE
+    assert lib.dl_read_error(h, None, 0, None) == dl.DL_ERR_INVALID_ARG
+    assert lib.dl_destroy_pool(h) == dl.DL_OK
+    assert lib.dl_destroy_pool(None) == dl.DL_ERR_INVALID_ARG
+
+
+def test_eager_only_pool_rejects_log_operations():
+    lib = dl.library()
+    st, h = _create(_desc(log=None, log_len=None, arrive=None))
+    P = 0x60000
+    a = dl.dl_step_args(P, 1, P, P, P, 1, P, 0, P, P)
+    assert lib.dl_decode_step(h, 0, ctypes.byref(a), 1, None) == dl.DL_ERR_UNSUPPORTED
+    assert lib.dl_append(h, 0, ctypes.byref(a), None) == dl.DL_ERR_UNSUPPORTED
+    assert lib.dl_merge(h, 0, P, 1, None) == dl.DL_ERR_UNSUPPORTED
+    assert lib.dl_materialize(h, 0, P, 1, P, None) == dl.DL_ERR_UNSUPPORTED
+    assert lib.dl_reset_slots(h, P, 1, None) == dl.DL_OK
+    lib.dl_destroy_pool(h)
+
+
+def test_status_strings():
+    for s in range(7):
+        assert dl.dl_status_string(s) and dl.dl_status_string(s) != "unknown status"
+    assert dl.dl_status_string(99) == "unknown status"

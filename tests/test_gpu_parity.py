@@ -1,0 +1,277 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, and the
+deferred path against the in-library eager path.  Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+from recurrent_state_serving_b200 import deltalog as dl
+from recurrent_state_serving_b200 import synth
+from recurrent_state_serving_b200.runner import DecodeRunner
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+# Reduced sizes: several heads and value tiles, odd batch sizes, non-contiguous slot
+# ids in a larger pool, and 256 steps (so every log fill level and many merges occur).
+REDUCED = {
+    "tiny_la": synth.TINY_LA,
+    "gla_L4": synth.GLA_DIAG.with_(batch=5, n_heads=3, n_kheads=3, log_cap=4),
+    "gla_L8": synth.GLA_DIAG.with_(batch=5, n_heads=3, n_kheads=3, log_cap=8),
+    "gla_L16": synth.GLA_DIAG.with_(batch=3, n_heads=3, n_kheads=3, log_cap=16),
+    "gla_L32": synth.GLA_DIAG.with_(batch=3, n_heads=3, n_kheads=3, log_cap=32),
+    "gdn_gva": synth.GDN_GVA,
+    "gdn_gva_256": synth.GDN_GVA.with_(batch=3, steps=256),
+    "kda": synth.KDA.with_(n_layers=2, batch=3, n_heads=4, n_kheads=4, steps=256),
+    "retnet": synth.RETNET.with_(n_layers=2, batch=7, n_heads=4, n_kheads=4, steps=256),
+}
+
+
+def _run_case(wl, update=None, slot_seed=0, extra_slots=3, tile_v=0):
+    T = wl.steps
+    ck = sorted({0, 1, T // 2, T})
+    r = DecodeRunner(wl, n_slots=wl.batch + extra_slots, slot_seed=slot_seed, update=update,
+                     tile_v=tile_v)
+    outs, states, _ = H.gpu_rollout(r, T, ckpts=ck)
+    assert r.errors() == 0
+    for layer in r.layers:
+        O, S = H.oracle_reference(wl, layer, T, ckpts=ck, update=update)
+        H.check_steps(outs[layer], O, what=f"{wl.name} layer {layer} output")
+        H.check_steps(states[layer], S, elem=None, what=f"{wl.name} layer {layer} state")
+    return r, outs
+
+
+@pytest.mark.parametrize("tile_v", [16, 32])
+@pytest.mark.parametrize("name", sorted(REDUCED))
+def test_parity_vs_oracle(name, tile_v):
+    wl = REDUCED[name]
+    if tile_v == 32 and (wl.d_k < 64 or wl.d_v % 32):
+        pytest.skip("32-wide value tiles need d_k >= 64 and d_v % 32 == 0")
+    _run_case(wl, tile_v=tile_v)
+
+
+def test_parity_delta_undecayed_reading():
+    _run_case(synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=96),
+              update="delta_undecayed")
+    _run_case(synth.GDN_GVA.with_(batch=2, steps=96), update="delta_undecayed")
+
+
+@pytest.mark.parametrize("shape", [(64, 80), (64, 64), (128, 256), (16, 48), (128, 48)])
+def test_parity_other_head_shapes(shape):
+    dk, dv = shape
+    wl = synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=2, d_k=dk, d_v=dv,
+                         steps=40, log_cap=6, qkv_std=1 / np.sqrt(dk))
+    tiles = [16, 32] if dk >= 64 and dv % 32 == 0 else [16]
+    for tv in tiles:
+        _run_case(wl, tile_v=tv)
+        _run_case(synth.GLA_DIAG.with_(batch=3, n_heads=2, n_kheads=1, d_k=dk, d_v=dv, steps=40,
+                                       log_cap=5, qkv_std=1 / np.sqrt(dk)), tile_v=tv)
+
+
+@pytest.mark.parametrize("name", ["tiny_la", "gla_L8", "gla_L32", "gdn_gva_256", "kda", "retnet"])
+def test_deferred_matches_eager_on_gpu(name):
+    wl = REDUCED[name]
+    T = wl.steps
+    tv = 32 if wl.d_k >= 64 else 16
+    rd = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, tile_v=tv)
+    re = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, mode="eager", tile_v=16)
+    od, sd, _ = H.gpu_rollout(rd, T, ckpts=[T])
+    oe, se, _ = H.gpu_rollout(re, T, ckpts=[T])
+    assert rd.errors() == 0 and re.errors() == 0
+    for layer in rd.layers:
+        H.check_steps(od[layer], oe[layer], tol=H.REL_L2_GPU, elem=None, what="deferred vs eager")
+        H.check_steps(sd[layer], se[layer], tol=H.REL_L2_GPU, elem=None, what="state")
+
+
+def test_log_cap_one_is_eager_bit_for_bit():
+    wl = synth.KDA.with_(n_layers=1, batch=4, n_heads=4, n_kheads=4, steps=24, log_cap=1)
+    rd = DecodeRunner(wl)
+    re = DecodeRunner(wl, mode="eager")
+    od, sd, _ = H.gpu_rollout(rd, wl.steps, ckpts=[wl.steps])
+    oe, se, _ = H.gpu_rollout(re, wl.steps, ckpts=[wl.steps])
+    np.testing.assert_array_equal(od[0], oe[0])
+    np.testing.assert_array_equal(sd[0], se[0])
+    assert int(rd.pool.log_len.abs().sum()) == 0
+
+
+def test_log_contents_match_the_deferred_oracle():
+    """Entry i of the ring holds (a_i, b_i, Lambda_i) exactly as the paper's log does."""
+    from oracle.deferred import DeferredHead
+    wl = synth.KDA.with_(n_layers=1, batch=2, n_heads=2, n_kheads=2, steps=11, log_cap=8)
+    r = DecodeRunner(wl)
+    _, _, inputs = H.gpu_rollout(r, wl.steps, keep_inputs=True)
+    S0 = synth.initial_state(wl, 0)
+    log = r.pool.log.double().cpu().numpy()
+    live = r.pool.log_len.cpu().numpy()
+    f = lambda x: synth.input_to_f64(x, wl.in_dtype)
+    dk, dv = wl.d_k, wl.d_v
+    for b in range(wl.batch):
+        s = r.slot_ids[b]
+        for h in range(wl.n_heads):
+            ref = DeferredHead(S0[b, h], wl.log_cap, wl.decay, wl.update)
+            for x in inputs[0]:
+                ref.decode(f(x["q"][b, h]), f(x["k"][b, h]), f(x["v"][b, h]),
+                           x["lam"][b, h], x["beta"][b, h])
+            assert live[s, 0] == ref.live == 11 - 8
+            for i in range(ref.live):
+                ent = log[s, 0, h, i]
+                np.testing.assert_allclose(ent[:dk], ref.K_log[i], rtol=0, atol=0)
+                assert H.rel_l2(ent[dk:dk + dv], ref.U_log[i]) < 1e-5
+                np.testing.assert_allclose(ent[dk + dv:], ref.Lam_log[i], rtol=1e-5, atol=1e-7)
+
+
+def test_append_then_merge_flow():
+    """dl_append fills all L rows, dl_merge folds them, decode continues."""
+    wl = synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=30, log_cap=5)
+    r = DecodeRunner(wl, n_slots=6, slot_seed=3)
+    r.load_initial_state()
+    T = wl.steps
+    gpu_states = []
+    for t in range(T):
+        x = r.gen_inputs(t, 0)
+        if t < 2 * wl.log_cap:   # append-only phase with explicit merges
+            dl.dl_append(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"])
+            if (t + 1) % wl.log_cap == 0:
+                assert int(r.pool.log_len[r.slots.long(), 0].min()) == wl.log_cap
+                dl.dl_merge(r.pool, 0, r.slots)
+        else:
+            r.call(0, x)
+        gpu_states.append(r.materialize(0).double().cpu().numpy())
+    assert r.errors() == 0
+    _, S = H.oracle_reference(wl, 0, T, ckpts=list(range(1, T + 1)))
+    H.check_steps(np.stack(gpu_states), S, elem=None, what="state")
+
+
+def test_materialize_leaves_pool_unchanged():
+    wl = synth.GLA_DIAG.with_(batch=3, n_heads=2, n_kheads=2, steps=5, log_cap=8)
+    r = DecodeRunner(wl)
+    H.gpu_rollout(r, wl.steps)
+    before = [t.clone() for t in (r.pool.state, r.pool.log, r.pool.log_len, r.pool.arrive)]
+    r.materialize(0)
+    torch.cuda.synchronize()
+    for a, b in zip(before, (r.pool.state, r.pool.log, r.pool.log_len, r.pool.arrive)):
+        assert torch.equal(a, b)
+
+
+def test_empty_batch_is_a_noop():
+    wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=1)
+    r = DecodeRunner(wl)
+    r.load_initial_state()
+    snap = r.pool.state.clone()
+    x = r.gen_inputs(0, 0)
+    empty = torch.zeros(0, dtype=torch.int32, device="cuda")
+    e = lambda t: t[:0].contiguous()
+    out = dl.dl_decode_step(r.pool, 0, empty, e(x["q"]), e(x["k"]), e(x["v"]), lam=e(x["lam"]))
+    dl.dl_merge(r.pool, 0, empty)
+    dl.dl_reset_slots(r.pool, empty)
+    assert out.shape == (0, 2, 128)
+    assert torch.equal(snap, r.pool.state) and r.errors() == 0
+
+
+def test_out_of_range_slot_sets_error_and_spares_others():
+    wl = synth.GLA_DIAG.with_(batch=3, n_heads=2, n_kheads=2, steps=3, log_cap=4)
+    good = DecodeRunner(wl)
+    og, _, _ = H.gpu_rollout(good, wl.steps)
+    bad = DecodeRunner(wl)
+    bad.load_initial_state()
+    slots = bad.slots.clone()
+    slots[1] = 99
+    outs = []
+    for t in range(wl.steps):
+        x = bad.gen_inputs(t, 0)
+        outs.append(bad.call(0, x, slots=slots).double().cpu().numpy())
+    assert bad.errors() & dl.DL_EBIT_SLOT_RANGE
+    assert bad.errors() == 0          # cleared by the previous read
+    o = np.stack(outs)
+    np.testing.assert_array_equal(o[:, [0, 2]], og[0][:, [0, 2]])
+
+
+def test_eager_step_on_live_log_is_refused():
+    wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=2, log_cap=4)
+    r = DecodeRunner(wl)
+    H.gpu_rollout(r, 2)
+    snap = r.pool.state.clone()
+    x = r.gen_inputs(5, 0)
+    dl.dl_eager_step(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"])
+    assert r.errors() == dl.DL_EBIT_LIVE_LOG
+    assert torch.equal(snap, r.pool.state)
+
+
+def test_full_log_without_auto_merge_is_refused():
+    wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=1, log_cap=3)
+    r = DecodeRunner(wl)
+    r.load_initial_state()
+    for t in range(3):
+        x = r.gen_inputs(t, 0)
+        dl.dl_decode_step(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], auto_merge=False)
+    assert r.errors() == 0
+    assert r.pool.log_len[r.slots.long(), 0].tolist() == [3, 3]
+    snap = r.pool.log.clone()
+    x = r.gen_inputs(3, 0)
+    dl.dl_decode_step(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], auto_merge=False)
+    assert r.errors() == dl.DL_EBIT_LOG_FULL
+    assert torch.equal(snap, r.pool.log)
+    # with auto-merge the same call folds the full log and the token into the base
+    o = dl.dl_decode_step(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"])
+    assert r.errors() == 0 and r.pool.log_len[r.slots.long(), 0].tolist() == [0, 0]
+    O, _ = H.oracle_reference(wl, 0, 4)
+    H.check_steps(o.double().cpu().numpy()[None], O[3:4])
+
+
+def test_reset_slots_empties_the_log_only():
+    wl = synth.GLA_DIAG.with_(batch=3, n_heads=2, n_kheads=2, steps=3, log_cap=8)
+    r = DecodeRunner(wl)
+    H.gpu_rollout(r, 3)
+    base = r.pool.state.clone()
+    dl.dl_reset_slots(r.pool, r.slots[:2].contiguous())
+    torch.cuda.synchronize()
+    assert r.pool.log_len[r.slots.long(), 0].tolist() == [0, 0, 3]
+    assert torch.equal(base, r.pool.state)
+    dense = r.materialize(0)
+    assert torch.equal(dense[0], base[r.slot_ids[0], 0])
+
+
+def test_lambda_per_head_diag_and_scalar():
+    for decay in ("scalar", "diag"):
+        wl = synth.RETNET.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=70, decay=decay,
+                                staggered=False, log_cap=8)
+        _run_case(wl)
+
+
+# --------------------------------------------------------------------------------
+# full sizes, in the launch configuration the benchmark times
+# --------------------------------------------------------------------------------
+def test_fullsize_gla_all_heads():
+    wl = synth.GLA_DIAG
+    r = DecodeRunner(wl)
+    outs, states, _ = H.gpu_rollout(r, wl.steps, ckpts=[wl.steps])
+    assert r.errors() == 0
+    O, S = H.oracle_reference(wl, 0, wl.steps, ckpts=[wl.steps])
+    H.check_steps(outs[0], O)
+    H.check_steps(states[0], S, elem=None)
+
+
+def test_fullsize_kda_sampled_rows():
+    wl = synth.KDA
+    rows = np.array([0, 77, 160, 255])
+    layers = [0, wl.n_layers - 1]
+    r = DecodeRunner(wl, layers=layers)
+    outs, _, kept = H.gpu_rollout(r, wl.steps, keep_inputs=True)
+    assert r.errors() == 0
+    for l in layers:
+        O, _ = H.oracle_reference(wl, l, wl.steps, rows=rows, main_inputs=kept[l])
+        H.check_steps(outs[l][:, rows], O)
+    del r
+    torch.cuda.empty_cache()
+
+
+def test_fullsize_retnet_b1024_sampled_rows():
+    wl = synth.RETNET.with_(batch=1024)
+    T = 40
+    rows = np.array([1, 500, 1023])
+    r = DecodeRunner(wl, layers=[3])
+    outs, _, kept = H.gpu_rollout(r, T, keep_inputs=True)
+    assert r.errors() == 0
+    O, _ = H.oracle_reference(wl, 3, T, rows=rows, main_inputs=kept[3])
+    H.check_steps(outs[3][:, rows], O)
+    del r
+    torch.cuda.empty_cache()
