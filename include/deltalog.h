@@ -82,6 +82,8 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
 #define DL_EBIT_LOG_FULL 0x2    /* append / decode without auto-merge on a full log   */
 #define DL_EBIT_LIVE_LOG 0x4    /* eager step on a slot whose log is not empty        */
 #define DL_EBIT_LOG_LEN 0x8     /* a stored live-log length outside [0, log_cap]     */
+#define DL_EBIT_TIMEOUT 0x10    /* a pipeline wait inside a kernel ran out of time and
+                                   the kernel abandoned the call (a library fault)    */
 
 /* Pool descriptor.  One pool covers n_slots request slots x n_layers
  * linear-attention layers x n_heads value heads.
@@ -103,9 +105,13 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
  *           per call.  Must be zero when the pool is created; the library returns
  *           them to zero at the end of every call.  Required with a log.
  *  err_word [1] int32 sticky device error bits; zero it before first use.
- *  tile_v   value-tile width B_V of a work unit (Section 3.3): 16 or 32 columns,
- *           or 0 to choose per launch (32 unless that leaves fewer than two CTAs
- *           per SM).  32 needs d_k >= 64 and d_v a multiple of 32.
+ *  tile_v   value-tile width B_V of a work unit (Section 3.3): 16 or 32 columns;
+ *           128 for whole-head work units run by the persistent, TMA-staged decode
+ *           kernel (needs d_k = d_v = 128 and log_cap <= 32; other calls of such a
+ *           pool use 16/32-wide tiles); 0 to choose per launch (whole heads for
+ *           d_k = d_v = 128, log_cap <= 32 and at least two heads per CTA slot,
+ *           else 32 columns unless that leaves SMs idle, else 16).  32 needs
+ *           d_k >= 64 and d_v a multiple of 32.
  *
  * The cumulative log-decay lbar of a slot is not stored separately: it equals
  * Lambda of the newest live entry (0 when the log is empty).

@@ -43,8 +43,17 @@ dl::KParams base_params(const dl_pool_desc &d, int layer) {
 }
 
 void set_tiles(const dl_pool_desc &d, dl::KParams &p, int batch, int &bv) {
-    bv = d.tile_v ? d.tile_v : dl::pick_bv(p.dk, p.dv, (long long)batch * p.H * (p.dv / 32));
+    bv = (d.tile_v == 16 || d.tile_v == 32) ? d.tile_v
+                                           : dl::pick_bv(p.dk, p.dv, (long long)batch * p.H * (p.dv / 32));
     p.nv = p.dv / bv;
+}
+
+// Full-head work units (persistent kernel) for a decode or eager step?
+bool use_persistent(const dl_pool_desc &d, int batch, bool want_out) {
+    if (!want_out || !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return false;
+    if (d.tile_v == 128) return true;
+    if (d.tile_v != 0) return false;
+    return (long long)batch * d.n_heads >= 2LL * dl::device_sm_count();
 }
 
 dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, bool need_out) {
@@ -83,11 +92,17 @@ dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_o
     p.eager = eager ? 1 : 0;
     p.want_out = want_out ? 1 : 0;
     p.undecayed = d.update == DL_UPDATE_DELTA_UNDECAYED ? 1 : 0;
-    int bv = 32;
-    set_tiles(d, p, a->batch, bv);
-    const cudaError_t e = dl::launch_step(p, bv, d.decay, d.update != DL_UPDATE_ADD,
-                                          a->in_dtype == DL_BF16,
-                                          static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (use_persistent(d, a->batch, want_out)) {
+        p.nv = 1;
+        e = dl::launch_persistent(p, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
+                                  static_cast<cudaStream_t>(stream));
+    } else {
+        int bv = 32;
+        set_tiles(d, p, a->batch, bv);
+        e = dl::launch_step(p, bv, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
+                            static_cast<cudaStream_t>(stream));
+    }
     return e == cudaSuccess ? DL_OK : DL_ERR_CUDA;
 }
 
@@ -103,8 +118,9 @@ DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
     if (!dk_supported(d.d_k)) return DL_ERR_SHAPE;
     if (d.d_v < 16 || d.d_v > 1024 || d.d_v % 16) return DL_ERR_SHAPE;
     if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
-    if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32) return DL_ERR_SHAPE;
+    if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32 && d.tile_v != 128) return DL_ERR_SHAPE;
     if (d.tile_v == 32 && (d.d_k < 64 || d.d_v % 32)) return DL_ERR_SHAPE;
+    if (d.tile_v == 128 && !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return DL_ERR_SHAPE;
     if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;

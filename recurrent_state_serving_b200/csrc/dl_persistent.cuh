@@ -1,0 +1,450 @@
+// Persistent, TMA-staged decode step for d_k = d_v = 128 (the shape of every
+// workload in the DeltaLog evaluation: H = 32 heads of 128 x 128 fp32 state).
+//
+// Work unit = one (slot, head): the whole 64 KB base state of a head, so the
+// key-side replay coefficients (DeltaLog paper, Section 3.3: "computed once per
+// slot-head pair") are formed once and the single owner of the shared log
+// metadata is the unit itself.  The grid is two CTAs per SM, each looping over
+// heads (blockIdx.x, + gridDim.x, ...).
+//
+// Warp roles inside a CTA:
+//  * producer warp: reads the slot id and live-log length of the next heads,
+//    prefetches their live log entries and token rows into L2, and streams each
+//    head's base state in four contiguous 16 KB chunks (32 rows x 128 columns)
+//    into a ring of shared-memory stages with cp.async.bulk (TMA bulk copies,
+//    evict-first in L2), completing on per-stage mbarriers.
+//  * 8 consumer warps: token prescale and ReplayPrep coefficients, the two
+//    mat-vecs S^T qt and S^T kt over the staged chunks, the value-log replay,
+//    b_t and o_t, the log append -- or, on the slot's merge step, the write-back
+//    of the materialised state straight from the staged chunks.
+// Stages are released per chunk on append heads and after the write-back on
+// merge heads, so HBM streaming continues while consumers do the per-head work.
+//
+// Every pipeline wait is bounded (100 ms); on expiry the CTA sets
+// DL_EBIT_TIMEOUT, stops, and waits (bounded again) for its own copies still in
+// flight before it exits.  Consumers take every wait decision jointly (a named
+// barrier with an OR reduction), so they never split across barriers.
+#pragma once
+
+#include "dl_kernels.cuh"
+#include "dl_ptx.cuh"
+
+namespace dl {
+namespace pk {
+
+constexpr int DK = 128, DV = 128;
+constexpr int CROWS = 32;                        // rows per chunk
+constexpr int NCHUNK = DK / CROWS;               // chunks per head
+constexpr int CFLOATS = CROWS * DV;              // floats per chunk
+constexpr uint32_t CBYTES = CFLOATS * 4;         // 16 KB
+constexpr int NCW = 8;                           // consumer warps
+constexpr int NCT = NCW * 32;                    // consumer threads
+constexpr int NTHREADS = NCT + 32;               // + producer warp
+constexpr int RPW = CROWS / NCW;                 // rows per consumer warp per chunk
+constexpr int LMAX = 32;                         // log capacity supported here
+constexpr int EPW = LMAX / NCW;                  // log entries per warp in ReplayPrep
+constexpr int PB = 8;                            // producer look-ahead batch (heads)
+constexpr uint64_t WAIT_NS = 100000000ull;       // bound on every pipeline wait
+constexpr int BAR_CONS = 1;                      // named barrier of the consumer warps
+
+// Byte offsets inside the dynamic shared-memory block.
+struct Layout {
+    size_t stages, A, b, red, vec, bt, cq, ck, idesc, flags, bars, total;
+    __host__ __device__ Layout(int ns, int L) {
+        const size_t L4 = (size_t)((L + 3) & ~3);
+        size_t o = 0;
+        stages = o; o += (size_t)ns * CBYTES;
+        A = o;      o += (size_t)L * DK * 4;      // A'_i rows of the merge step
+        b = o;      o += (size_t)L * DV * 4;      // b_i of the live entries
+        red = o;    o += (size_t)2 * NCW * DV * 4;
+        vec = o;    o += (size_t)7 * DK * 4;      // q, k, qt, kt, lbar_t, lbar_{t-1}, e^{lbar_t}
+        bt = o;     o += (size_t)DV * 4;
+        cq = o;     o += L4 * 4;
+        ck = o;     o += L4 * 4;
+        idesc = o;  o += (size_t)ns * 16;
+        flags = o;  o += 16;
+        bars = o;   o += (size_t)2 * ns * 8;
+        total = o;
+    }
+};
+
+__device__ __forceinline__ float4 ldg4(const float *p) {
+    return __ldg(reinterpret_cast<const float4 *>(p));
+}
+
+template <int DECAY, bool DELTA, typename IT>
+__global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KParams p)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int NS = p.ns;
+    const Layout lay(NS, p.L);
+    float *stages = reinterpret_cast<float *>(smem + lay.stages);
+    float *s_A = reinterpret_cast<float *>(smem + lay.A);
+    float *s_b = reinterpret_cast<float *>(smem + lay.b);
+    float *s_red = reinterpret_cast<float *>(smem + lay.red);
+    float *s_q = reinterpret_cast<float *>(smem + lay.vec);
+    float *s_k = s_q + DK, *s_qt = s_k + DK, *s_kt = s_qt + DK;
+    float *s_ell = s_kt + DK, *s_ellp = s_ell + DK, *s_e = s_ellp + DK;
+    float *s_bt = reinterpret_cast<float *>(smem + lay.bt);
+    float *s_cq = reinterpret_cast<float *>(smem + lay.cq);
+    float *s_ck = reinterpret_cast<float *>(smem + lay.ck);
+    int4 *idesc = reinterpret_cast<int4 *>(smem + lay.idesc);
+    volatile int *flags = reinterpret_cast<volatile int *>(smem + lay.flags);
+    float *s_kq = reinterpret_cast<float *>(smem + lay.flags) + 3;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+    uint64_t *empty = full + NS;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_items = p.batch * p.H;
+    const int G = gridDim.x;
+    const int E = p.E;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], NCW);
+        }
+        flags[0] = 0;  // abort
+        flags[1] = 0;  // chunks issued
+        flags[2] = 0;  // chunks waited by the consumers
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == NCW) {
+        // ------------------------------------------------------------------ producer
+        const uint64_t pol = ptx::policy_evict_first();
+        int g = 0, n = 0;
+        bool abort = false;
+        for (int base = blockIdx.x; base < n_items && !abort; base += PB * G) {
+            const int it = base + lane * G;
+            int s = -1, c = 0, st = 0;
+            if (lane < PB && it < n_items) {
+                const int bi = it / p.H, h = it % p.H;
+                s = p.slots[bi];
+                if (s < 0 || s >= p.n_slots) {
+                    st = DL_EBIT_SLOT_RANGE;
+                } else {
+                    const size_t sl = (size_t)s * p.n_layers + p.layer;
+                    c = p.log_len ? p.log_len[sl] : 0;
+                    if (p.eager) {
+                        if (c != 0) st = DL_EBIT_LIVE_LOG;
+                    } else if (c < 0 || c > p.L) {
+                        st = DL_EBIT_LOG_LEN;
+                    } else if (!(p.auto_merge && c >= p.L - 1) && c >= p.L) {
+                        st = DL_EBIT_LOG_FULL;
+                    }
+                }
+                if (st == 0) {  // warm L2 with what the consumers will read for this head
+                    const size_t head = ((size_t)s * p.n_layers + p.layer) * p.H + h;
+                    if (c > 0) ptx::prefetch_l2_aligned(p.log + head * (size_t)p.L * E, (uint32_t)(c * E * 4));
+                    const int gk = h / (p.H / p.Hk);
+                    const IT *qrow = static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + gk) * DK;
+                    const IT *krow = static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + gk) * DK;
+                    ptx::prefetch_l2_aligned(qrow, DK * sizeof(IT));
+                    ptx::prefetch_l2_aligned(krow, DK * sizeof(IT));
+                    ptx::prefetch_l2_aligned(static_cast<const IT *>(p.v) + ((size_t)bi * p.H + h) * DV,
+                                     DV * sizeof(IT));
+                    if (DECAY == DL_DECAY_DIAG && !p.lam_const)
+                        ptx::prefetch_l2_aligned(p.lam + ((size_t)bi * p.H + h) * DK, DK * 4);
+                }
+            }
+            for (int k = 0; k < PB; ++k) {
+                const int itk = base + k * G;
+                if (itk >= n_items) break;
+                const int sk = __shfl_sync(0xffffffffu, s, k);
+                const int ck = __shfl_sync(0xffffffffu, c, k);
+                const int stk = __shfl_sync(0xffffffffu, st, k);
+                if (lane == 0) {
+                    if (stk) atomicOr(p.err, stk);
+                    const int bi = itk / p.H, h = itk % p.H;
+                    const size_t head = stk ? 0 : ((size_t)sk * p.n_layers + p.layer) * p.H + h;
+                    const float *tile = p.state + head * (size_t)(DK * DV);
+                    const int merge_now = p.eager || (p.auto_merge && ck >= p.L - 1);
+                    const int nch = stk ? 1 : NCHUNK;
+                    (void)bi;
+                    for (int q = 0; q < nch; ++q, ++g) {
+                        const int sg = g % NS;
+                        if (!ptx::mbar_wait_bounded(&empty[sg], ((g / NS) & 1) ^ 1, WAIT_NS)) {
+                            abort = true;
+                            break;
+                        }
+                        if (q == 0) idesc[n % NS] = make_int4(sk, ck, stk == 0, merge_now);
+                        if (stk) {
+                            ptx::mbar_arrive(&full[sg]);
+                        } else {
+                            ptx::mbar_arrive_expect_tx(&full[sg], CBYTES);
+                            ptx::bulk_g2s(stages + (size_t)sg * CFLOATS, tile + (size_t)q * CFLOATS,
+                                          CBYTES, &full[sg], pol);
+                        }
+                    }
+                    ++n;
+                }
+                abort = __shfl_sync(0xffffffffu, abort, 0);
+                if (abort) break;
+            }
+        }
+        if (lane == 0) {
+            flags[1] = g;
+            if (abort) {
+                flags[0] = 1;
+                atomicOr(p.err, DL_EBIT_TIMEOUT);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ consumers
+        const int t = tid;
+        int g = 0, gw = 0, n = 0;
+        bool abort = false;
+        for (int it = blockIdx.x; it < n_items; it += G, ++n) {
+            {
+                const bool ok = ptx::mbar_wait_bounded(&full[g % NS], (g / NS) & 1, WAIT_NS);
+                if (ptx::bar_or(BAR_CONS, NCT, !ok)) {
+                    abort = true;
+                    break;
+                }
+                ++gw;
+            }
+            const int4 d = idesc[n % NS];
+            if (!d.z) {  // skipped head: one empty stage was sent
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[g % NS]);
+                ++g;
+                continue;
+            }
+            const int s = d.x, c = d.y;
+            const bool merge_now = d.w != 0;
+            const int bi = it / p.H, h = it % p.H;
+            const size_t sl = (size_t)s * p.n_layers + p.layer;
+            const size_t head = sl * p.H + h;
+            float *tile = p.state + head * (size_t)(DK * DV);
+            float *ring = p.log ? p.log + head * (size_t)p.L * E : nullptr;
+            const size_t row = (size_t)bi * p.H + h;
+
+            // -- A. issue this head's loads: log keys/snapshots, token, log values
+            float4 Areg[EPW], Lreg[EPW];
+#pragma unroll
+            for (int k = 0; k < EPW; ++k) {
+                const int i = warp + NCW * k;
+                Areg[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                Lreg[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (i < c) {
+                    const float *ent = ring + (size_t)i * E;
+                    Areg[k] = ldg4(ent + 4 * lane);
+                    if (DECAY == DL_DECAY_DIAG) Lreg[k] = ldg4(ent + DK + DV + 4 * lane);
+                    if (DECAY == DL_DECAY_SCALAR) Lreg[k].x = __ldg(ent + DK + DV);
+                }
+            }
+            float vv = 0.f, bb = 0.f;
+            if (t < DK) {
+                const int r = t;
+                const int gk = h / (p.H / p.Hk);
+                const float qv = to_f32(static_cast<const IT *>(p.q)[((size_t)bi * p.Hk + gk) * DK + r]);
+                const float kv = to_f32(static_cast<const IT *>(p.k)[((size_t)bi * p.Hk + gk) * DK + r]);
+                vv = to_f32(static_cast<const IT *>(p.v)[row * DV + r]);
+                if (DELTA) bb = p.beta[row];
+                float lp = 0.f, lt = 0.f, et = 1.f, ek = 1.f;
+                if (DECAY == DL_DECAY_DIAG) {
+                    lp = c > 0 ? __ldg(ring + (size_t)(c - 1) * E + DK + DV + r) : 0.f;
+                    lt = lp + (p.lam_const ? p.lam[(size_t)h * DK + r] : p.lam[row * DK + r]);
+                } else if (DECAY == DL_DECAY_SCALAR) {
+                    lp = c > 0 ? __ldg(ring + (size_t)(c - 1) * E + DK + DV) : 0.f;
+                    lt = lp + (p.lam_const ? p.lam[h] : p.lam[row]);
+                }
+                if (DECAY != DL_DECAY_NONE) {
+                    et = expf(lt);
+                    ek = (DELTA && p.undecayed) ? expf(lp) : et;
+                }
+                s_q[r] = qv;
+                s_k[r] = kv;
+                s_ell[r] = lt;
+                s_ellp[r] = lp;
+                s_e[r] = et;
+                s_qt[r] = et * qv;
+                s_kt[r] = ek * kv;
+            } else {
+                constexpr int NB = NCT - DK;     // 128 threads stage b_i
+                const int nvec = c * (DV / 4);
+                for (int idx0 = t - DK; idx0 < nvec; idx0 += 4 * NB) {
+                    float4 tmp[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int idx = idx0 + u * NB;
+                        if (idx < nvec)
+                            tmp[u] = ldg4(ring + (size_t)(idx / (DV / 4)) * E + DK + 4 * (idx % (DV / 4)));
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int idx = idx0 + u * NB;
+                        if (idx < nvec) reinterpret_cast<float4 *>(s_b)[idx] = tmp[u];
+                    }
+                }
+            }
+            ptx::bar_sync(BAR_CONS, NCT);
+
+            // -- ReplayPrep: cq_i = sum_r a_i[r] e^{lbar_t[r]-Lambda_i[r]} q[r] (and ck_i)
+#pragma unroll
+            for (int k = 0; k < EPW; ++k) {
+                const int i = warp + NCW * k;
+                if (i < c) {
+                    const float av[4] = {Areg[k].x, Areg[k].y, Areg[k].z, Areg[k].w};
+                    const float Lv[4] = {Lreg[k].x, Lreg[k].y, Lreg[k].z, Lreg[k].w};
+                    float fs = 1.f, fk = 1.f;
+                    if (DECAY == DL_DECAY_SCALAR) {
+                        fs = expf(s_ell[0] - Lv[0]);
+                        fk = (DELTA && p.undecayed) ? expf(s_ellp[0] - Lv[0]) : fs;
+                    }
+                    float pq = 0.f, pk = 0.f;
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int r = 4 * lane + x;
+                        float w, wk;
+                        if (DECAY == DL_DECAY_DIAG) {
+                            w = av[x] * expf(s_ell[r] - Lv[x]);
+                            wk = (DELTA && p.undecayed) ? av[x] * expf(s_ellp[r] - Lv[x]) : w;
+                        } else {
+                            w = av[x] * fs;
+                            wk = av[x] * fk;
+                        }
+                        pq = fmaf(w, s_q[r], pq);
+                        if (DELTA) pk = fmaf(wk, s_k[r], pk);
+                        if (merge_now) s_A[i * DK + r] = w;
+                    }
+                    pq = warp_sum(pq);
+                    if (DELTA) pk = warp_sum(pk);
+                    if (lane == 0) {
+                        s_cq[i] = pq;
+                        s_ck[i] = pk;
+                    }
+                }
+            }
+            if (warp == NCW - 1) {  // a_t . q_t of the new entry
+                float x = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) x = fmaf(s_q[4 * lane + u], s_k[4 * lane + u], x);
+                x = warp_sum(x);
+                if (lane == 0) *s_kq = x;
+            }
+            ptx::bar_sync(BAR_CONS, NCT);
+
+            // -- AppendDecode: y_q = S^T qt, y_k = S^T kt over the staged chunks
+            float4 yq = make_float4(0.f, 0.f, 0.f, 0.f), yk = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < NCHUNK; ++q) {
+                const int gq = g + q, sg = gq % NS;
+                if (q > 0) {
+                    const bool ok = ptx::mbar_wait_bounded(&full[sg], (gq / NS) & 1, WAIT_NS);
+                    if (ptx::bar_or(BAR_CONS, NCT, !ok)) {
+                        abort = true;
+                        break;
+                    }
+                    ++gw;
+                }
+                const float *stg = stages + (size_t)sg * CFLOATS;
+#pragma unroll
+                for (int rr = 0; rr < RPW; ++rr) {
+                    const int rl = warp * RPW + rr, r = q * CROWS + rl;
+                    const float4 S = reinterpret_cast<const float4 *>(stg + rl * DV)[lane];
+                    fma4(yq, s_qt[r], S);
+                    if (DELTA) fma4(yk, s_kt[r], S);
+                }
+                if (!merge_now) {
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&empty[sg]);
+                }
+            }
+            if (abort) break;
+            reinterpret_cast<float4 *>(s_red + warp * DV)[lane] = yq;
+            reinterpret_cast<float4 *>(s_red + (NCW + warp) * DV)[lane] = yk;
+            ptx::bar_sync(BAR_CONS, NCT);
+
+            // -- value-log replay, b_t, o_t, append (Finalize commits the length below)
+            if (t < DV) {
+                float Yq = 0.f, Yk = 0.f;
+#pragma unroll
+                for (int w = 0; w < NCW; ++w) {
+                    Yq += s_red[w * DV + t];
+                    Yk += s_red[(NCW + w) * DV + t];
+                }
+                for (int i = 0; i < c; ++i) {
+                    const float b = s_b[i * DV + t];
+                    Yq = fmaf(b, s_cq[i], Yq);
+                    if (DELTA) Yk = fmaf(b, s_ck[i], Yk);
+                }
+                const float bt = DELTA ? bb * (vv - Yk) : vv;
+                if (p.want_out) p.out[row * DV + t] = fmaf(bt, *s_kq, Yq);
+                if (!merge_now) ring[(size_t)c * E + DK + t] = bt;
+                s_bt[t] = bt;
+            } else if (!merge_now) {
+                const int r = t - DV;
+                float *ent = ring + (size_t)c * E;
+                ent[r] = s_k[r];
+                if (DECAY == DL_DECAY_DIAG) ent[DK + DV + r] = s_ell[r];
+                if (DECAY == DL_DECAY_SCALAR && r == 0) ent[DK + DV] = s_ell[0];
+            }
+
+            // -- merge step: S_t = e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, from the stages
+            if (merge_now) {
+                ptx::bar_sync(BAR_CONS, NCT);
+                const float4 bt4 = reinterpret_cast<const float4 *>(s_bt)[lane];
+                for (int q = 0; q < NCHUNK; ++q) {
+                    const int sg = (g + q) % NS;
+                    const float *stg = stages + (size_t)sg * CFLOATS;
+                    float4 acc[RPW];
+#pragma unroll
+                    for (int rr = 0; rr < RPW; ++rr) {
+                        const int rl = warp * RPW + rr, r = q * CROWS + rl;
+                        const float4 S = reinterpret_cast<const float4 *>(stg + rl * DV)[lane];
+                        const float e = s_e[r];
+                        acc[rr] = make_float4(S.x * e, S.y * e, S.z * e, S.w * e);
+                        fma4(acc[rr], s_k[r], bt4);
+                    }
+                    for (int i = 0; i < c; ++i) {
+                        const float4 b4 = reinterpret_cast<const float4 *>(s_b + i * DV)[lane];
+#pragma unroll
+                        for (int rr = 0; rr < RPW; ++rr)
+                            fma4(acc[rr], s_A[i * DK + q * CROWS + warp * RPW + rr], b4);
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < RPW; ++rr) {
+                        const int r = q * CROWS + warp * RPW + rr;
+                        __stcs(reinterpret_cast<float4 *>(tile + (size_t)r * DV) + lane, acc[rr]);
+                    }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&empty[sg]);
+                }
+            }
+            g += NCHUNK;
+
+            // -- Finalize: after every consumer is done with this head, the last unit
+            //    of the (slot, layer) commits the live length
+            ptx::bar_sync(BAR_CONS, NCT);
+            if (t == 0 && !p.eager) {
+                __threadfence();
+                const int old = atomicAdd(p.arrive + sl, 1);
+                if (old == p.H - 1) {
+                    p.log_len[sl] = merge_now ? 0 : c + 1;
+                    p.arrive[sl] = 0;
+                }
+            }
+        }
+        if (t == 0) {
+            flags[2] = gw;
+            if (abort) {
+                flags[0] = 1;
+                atomicOr(p.err, DL_EBIT_TIMEOUT);
+            }
+        }
+    }
+
+    // Only after an abandoned wait can copies still be in flight: wait for them
+    // (bounded) so no bulk copy lands in shared memory after the CTA has exited.
+    __syncthreads();
+    if (tid == 0 && flags[0]) {
+        const int issued = flags[1], waited = flags[2];
+        for (int gg = waited; gg < issued; ++gg)
+            ptx::mbar_wait_bounded(&full[gg % NS], (gg / NS) & 1, WAIT_NS);
+    }
+}
+
+}  // namespace pk
+}  // namespace dl

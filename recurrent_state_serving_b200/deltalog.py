@@ -29,7 +29,8 @@ DL_OK, DL_ERR_INVALID_ARG, DL_ERR_SHAPE, DL_ERR_DTYPE, DL_ERR_UNSUPPORTED, DL_ER
 DECAY = {"none": 0, "scalar": 1, "diag": 2}
 UPDATE = {"add": 0, "delta": 1, "delta_undecayed": 2}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
-DL_EBIT_SLOT_RANGE, DL_EBIT_LOG_FULL, DL_EBIT_LIVE_LOG, DL_EBIT_LOG_LEN = 0x1, 0x2, 0x4, 0x8
+DL_EBIT_SLOT_RANGE, DL_EBIT_LOG_FULL, DL_EBIT_LIVE_LOG, DL_EBIT_LOG_LEN, DL_EBIT_TIMEOUT = \
+    0x1, 0x2, 0x4, 0x8, 0x10
 
 
 class dl_pool_desc(ctypes.Structure):

@@ -40,19 +40,28 @@ def _run_case(wl, update=None, slot_seed=0, extra_slots=3, tile_v=0):
     return r, outs
 
 
-@pytest.mark.parametrize("tile_v", [16, 32])
+def _tile_ok(wl, tile_v):
+    if tile_v == 32:
+        return wl.d_k >= 64 and wl.d_v % 32 == 0
+    if tile_v == 128:
+        return wl.d_k == 128 and wl.d_v == 128 and wl.log_cap <= 32
+    return True
+
+
+@pytest.mark.parametrize("tile_v", [16, 32, 128])
 @pytest.mark.parametrize("name", sorted(REDUCED))
 def test_parity_vs_oracle(name, tile_v):
     wl = REDUCED[name]
-    if tile_v == 32 and (wl.d_k < 64 or wl.d_v % 32):
-        pytest.skip("32-wide value tiles need d_k >= 64 and d_v % 32 == 0")
+    if not _tile_ok(wl, tile_v):
+        pytest.skip("tile width not applicable to this head shape")
     _run_case(wl, tile_v=tile_v)
 
 
-def test_parity_delta_undecayed_reading():
+@pytest.mark.parametrize("tile_v", [32, 128])
+def test_parity_delta_undecayed_reading(tile_v):
     _run_case(synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=96),
-              update="delta_undecayed")
-    _run_case(synth.GDN_GVA.with_(batch=2, steps=96), update="delta_undecayed")
+              update="delta_undecayed", tile_v=tile_v)
+    _run_case(synth.GDN_GVA.with_(batch=2, steps=96), update="delta_undecayed", tile_v=tile_v)
 
 
 @pytest.mark.parametrize("shape", [(64, 80), (64, 64), (128, 256), (16, 48), (128, 48)])
@@ -67,13 +76,18 @@ def test_parity_other_head_shapes(shape):
                                        log_cap=5, qkv_std=1 / np.sqrt(dk)), tile_v=tv)
 
 
+@pytest.mark.parametrize("tiles", [(32, 16), (128, 128), (128, 32)])
 @pytest.mark.parametrize("name", ["tiny_la", "gla_L8", "gla_L32", "gdn_gva_256", "kda", "retnet"])
-def test_deferred_matches_eager_on_gpu(name):
+def test_deferred_matches_eager_on_gpu(name, tiles):
     wl = REDUCED[name]
     T = wl.steps
-    tv = 32 if wl.d_k >= 64 else 16
-    rd = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, tile_v=tv)
-    re = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, mode="eager", tile_v=16)
+    td, te = tiles
+    if wl.d_k == 16:
+        if tiles != (32, 16):
+            pytest.skip("one tiling for d_k = 16")
+        td = 16
+    rd = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, tile_v=td)
+    re = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=1, mode="eager", tile_v=te)
     od, sd, _ = H.gpu_rollout(rd, T, ckpts=[T])
     oe, se, _ = H.gpu_rollout(re, T, ckpts=[T])
     assert rd.errors() == 0 and re.errors() == 0
@@ -82,10 +96,11 @@ def test_deferred_matches_eager_on_gpu(name):
         H.check_steps(sd[layer], se[layer], tol=H.REL_L2_GPU, elem=None, what="state")
 
 
-def test_log_cap_one_is_eager_bit_for_bit():
+@pytest.mark.parametrize("tile_v", [0, 16, 128])
+def test_log_cap_one_is_eager_bit_for_bit(tile_v):
     wl = synth.KDA.with_(n_layers=1, batch=4, n_heads=4, n_kheads=4, steps=24, log_cap=1)
-    rd = DecodeRunner(wl)
-    re = DecodeRunner(wl, mode="eager")
+    rd = DecodeRunner(wl, tile_v=tile_v)
+    re = DecodeRunner(wl, mode="eager", tile_v=tile_v)
     od, sd, _ = H.gpu_rollout(rd, wl.steps, ckpts=[wl.steps])
     oe, se, _ = H.gpu_rollout(re, wl.steps, ckpts=[wl.steps])
     np.testing.assert_array_equal(od[0], oe[0])
@@ -93,11 +108,12 @@ def test_log_cap_one_is_eager_bit_for_bit():
     assert int(rd.pool.log_len.abs().sum()) == 0
 
 
-def test_log_contents_match_the_deferred_oracle():
+@pytest.mark.parametrize("tile_v", [16, 128])
+def test_log_contents_match_the_deferred_oracle(tile_v):
     """Entry i of the ring holds (a_i, b_i, Lambda_i) exactly as the paper's log does."""
     from oracle.deferred import DeferredHead
     wl = synth.KDA.with_(n_layers=1, batch=2, n_heads=2, n_kheads=2, steps=11, log_cap=8)
-    r = DecodeRunner(wl)
+    r = DecodeRunner(wl, tile_v=tile_v)
     _, _, inputs = H.gpu_rollout(r, wl.steps, keep_inputs=True)
     S0 = synth.initial_state(wl, 0)
     log = r.pool.log.double().cpu().numpy()
@@ -167,11 +183,12 @@ def test_empty_batch_is_a_noop():
     assert torch.equal(snap, r.pool.state) and r.errors() == 0
 
 
-def test_out_of_range_slot_sets_error_and_spares_others():
+@pytest.mark.parametrize("tile_v", [0, 128])
+def test_out_of_range_slot_sets_error_and_spares_others(tile_v):
     wl = synth.GLA_DIAG.with_(batch=3, n_heads=2, n_kheads=2, steps=3, log_cap=4)
-    good = DecodeRunner(wl)
+    good = DecodeRunner(wl, tile_v=tile_v)
     og, _, _ = H.gpu_rollout(good, wl.steps)
-    bad = DecodeRunner(wl)
+    bad = DecodeRunner(wl, tile_v=tile_v)
     bad.load_initial_state()
     slots = bad.slots.clone()
     slots[1] = 99
@@ -185,9 +202,10 @@ def test_out_of_range_slot_sets_error_and_spares_others():
     np.testing.assert_array_equal(o[:, [0, 2]], og[0][:, [0, 2]])
 
 
-def test_eager_step_on_live_log_is_refused():
+@pytest.mark.parametrize("tile_v", [0, 128])
+def test_eager_step_on_live_log_is_refused(tile_v):
     wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=2, log_cap=4)
-    r = DecodeRunner(wl)
+    r = DecodeRunner(wl, tile_v=tile_v)
     H.gpu_rollout(r, 2)
     snap = r.pool.state.clone()
     x = r.gen_inputs(5, 0)
@@ -196,9 +214,10 @@ def test_eager_step_on_live_log_is_refused():
     assert torch.equal(snap, r.pool.state)
 
 
-def test_full_log_without_auto_merge_is_refused():
+@pytest.mark.parametrize("tile_v", [0, 128])
+def test_full_log_without_auto_merge_is_refused(tile_v):
     wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=1, log_cap=3)
-    r = DecodeRunner(wl)
+    r = DecodeRunner(wl, tile_v=tile_v)
     r.load_initial_state()
     for t in range(3):
         x = r.gen_inputs(t, 0)
@@ -230,18 +249,20 @@ def test_reset_slots_empties_the_log_only():
     assert torch.equal(dense[0], base[r.slot_ids[0], 0])
 
 
-def test_lambda_per_head_diag_and_scalar():
+@pytest.mark.parametrize("tile_v", [0, 128])
+def test_lambda_per_head_diag_and_scalar(tile_v):
     for decay in ("scalar", "diag"):
         wl = synth.RETNET.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=70, decay=decay,
                                 staggered=False, log_cap=8)
-        _run_case(wl)
+        _run_case(wl, tile_v=tile_v)
 
 
 # --------------------------------------------------------------------------------
 # full sizes, in the launch configuration the benchmark times
 # --------------------------------------------------------------------------------
-def test_fullsize_gla_all_heads():
-    wl = synth.GLA_DIAG
+@pytest.mark.parametrize("log_cap", synth.GLA_LOG_CAPS)
+def test_fullsize_gla_all_heads(log_cap):
+    wl = synth.GLA_DIAG.with_(log_cap=log_cap)
     r = DecodeRunner(wl)
     outs, states, _ = H.gpu_rollout(r, wl.steps, ckpts=[wl.steps])
     assert r.errors() == 0
