@@ -7,9 +7,11 @@
 A step is one decode step of the whole batch over all layers of the workload (one
 library call per layer), with every slot advancing by one token; merges happen on
 each slot's own merge step inside the same call.  Inputs are seeded synthetic
-tensors resident in HBM before timing starts.  L2 (126 MB) is flushed by writing a
-256 MiB buffer before every timed step, outside the timed interval; each step is
-bracketed by CUDA events on the launching stream.
+tensors resident in HBM before timing starts.  Before every timed step, outside the
+timed interval, L2 (126 MB) is flushed by writing a 256 MiB buffer and then reading
+a second 256 MiB buffer: the read evicts the dirty lines the write left, so their
+write-back is not charged to the timed kernel and it starts from a cold, clean L2.
+Each step is bracketed by CUDA events on the launching stream.
 
 Multi-GPU (torchrun, one process per GPU): the slots are independent, so each rank
 runs its own replica of the workload (weak scaling, no collective on the data
@@ -37,7 +39,16 @@ METRIC = "decode head-steps/s (batch x heads x layers)"
 UNIT = "head-steps/s"
 FLUSH_BYTES = 256 << 20
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "step_kernel_traffic.txt")
-KERNEL_SRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc", "dl_kernels.cuh")
+CSRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc")
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a recorded ncu traffic figure is only valid for it."""
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        h.update(f.encode())
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -52,6 +63,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--tile-v", type=int, default=0,
+                    help="work-unit width: 0 automatic, 16/32 value tiles, 128 whole heads")
     return ap.parse_args()
 
 
@@ -65,12 +78,13 @@ def workload(a):
     return wl
 
 
-def config_of(wl, n_gpus):
+def config_of(wl, n_gpus, tile_v=0):
     return {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}",
+            "tile_v": tile_v or "auto",
             "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
             "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
             "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
-            "l2": "flushed: 256 MiB write before every timed step, outside the timed interval",
+            "l2": "flushed before every timed step, outside the timed interval: 256 MiB write, then 256 MiB read of another buffer (evicts the dirty lines)",
             "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
 
 
@@ -92,8 +106,7 @@ def recorded_traffic(workload_key):
         if "=" in line and not line.lstrip().startswith("#"):
             k, v = line.split("=", 1)
             kv[k.strip()] = v.strip()
-    src_hash = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
-    if kv.get("kernel_sha") != src_hash or kv.get("workload") != workload_key:
+    if kv.get("kernel_sha") != kernel_source_hash() or kv.get("workload") != workload_key:
         return None
     try:
         return float(kv["dram_bytes_per_launch"])
@@ -165,6 +178,30 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------------
+def res_kernel_name(wl, tile_v):
+    whole = tile_v == 128 or (tile_v == 0 and wl.d_k == 128 and wl.d_v == 128 and wl.log_cap <= 32
+                              and wl.batch * wl.n_heads >= 2 * 148)
+    return "dl::pk::persistent_step_kernel" if whole else "dl::step_kernel"
+
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the timing rule for multi-GPU runs)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------
 def run_gpu(a, wl, rank, world, dist):
@@ -175,6 +212,12 @@ def run_gpu(a, wl, rank, world, dist):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        torch.sum(flush_rd, out=flush_sink)
     L, K, W = wl.log_cap, a.steps, a.warmup
     ndist = max(1, min(wl.steps, 256 // wl.n_layers))
 
@@ -185,11 +228,7 @@ def run_gpu(a, wl, rank, world, dist):
         torch.cuda.synchronize()
 
     def reduce_max(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(x, dist, dev)
 
     host_inputs = [[synth.step_inputs(wl, t, l) for l in range(wl.n_layers)] for t in range(ndist)]
     sampler = ClockSampler(dev.index)
@@ -204,7 +243,7 @@ def run_gpu(a, wl, rank, world, dist):
         t0 = time.time()
         evs = []
         for i in range(n_steps):
-            flush.zero_()
+            flush_l2()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -218,7 +257,7 @@ def run_gpu(a, wl, rank, world, dist):
         return ms
 
     # ---- deferred (the product path) ----
-    r = DecodeRunner(wl, device=str(dev))
+    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v)
     r.load_initial_state()
     r.run_presteps()
     dev_inputs = [[r.device_inputs(x) for x in per_layer] for per_layer in host_inputs]
@@ -237,8 +276,7 @@ def run_gpu(a, wl, rank, world, dist):
     assert r.errors() == 0, "device error bits set during the benchmark"
     total_ms = sum(ms)
     max_ms = reduce_max(total_ms)
-    units = wl.units_per_step * K * world
-    value = units / (max_ms / 1e3)
+    value = whole_job_rate(wl.units_per_step * K, world, max_ms)
 
     # algorithmic bytes of the timed launches: slot b enters timed step i with
     # c = (offset_b + W + i) mod L live entries (auto-merge cycle of length L)
@@ -256,7 +294,7 @@ def run_gpu(a, wl, rank, world, dist):
     roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved_gbs / peak, 4), "peak_source": peak_src,
             "traffic": dram, "algorithmic_bytes_per_launch": round(bytes_total / launches),
-            "kernel": "dl::step_kernel", "launches_timed": launches,
+            "kernel": res_kernel_name(wl, a.tile_v), "launches_timed": launches,
             "avg_launch_us": round(total_ms * 1e3 / launches, 3),
             "frac_of_8tbs_spec": round(achieved_gbs / 8000.0, 4)}
 
@@ -264,7 +302,7 @@ def run_gpu(a, wl, rank, world, dist):
 
     # ---- eager comparison (same workload, full read-modify-write each step) ----
     if not a.no_eager:
-        re_ = DecodeRunner(wl, device=str(dev), mode="eager")
+        re_ = DecodeRunner(wl, device=str(dev), mode="eager", tile_v=a.tile_v)
         re_.load_initial_state()
         prep_e = [[dl.PreparedStep("eager", re_.pool, l, re_.slots, x["q"], x["k"], x["v"], x["lam"],
                                    x["beta"], outs[l], wl.lambda_const) for l, x in enumerate(per_layer)]
@@ -274,7 +312,7 @@ def run_gpu(a, wl, rank, world, dist):
         assert re_.errors() == 0
         tot_e = reduce_max(sum(ms_e))
         eb = traffic.eager_head_step(wl) * wl.units_per_step * K
-        result["eager"] = {"value": wl.units_per_step * K * world / (tot_e / 1e3),
+        result["eager"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_e),
                            "ms_per_step": tot_e / K,
                            "algorithmic_bytes_per_step": round(eb / K),
                            "achieved_gbs": round(eb / (sum(ms_e) / 1e3) / 1e9, 1)}
@@ -310,7 +348,7 @@ def run_gpu(a, wl, rank, world, dist):
         ms_2 = timed(r, e2e_calls, K)
         assert r.errors() == 0
         tot_2 = reduce_max(sum(ms_2))
-        result["e2e"] = {"value": wl.units_per_step * K * world / (tot_2 / 1e3), "unit": UNIT,
+        result["e2e"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_2), "unit": UNIT,
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "ms_per_step": tot_2 / K,
                          "path": "pinned host inputs -> H2D copy -> dl_decode_step per layer -> D2H of o_t, all inside the events"}
@@ -435,7 +473,7 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; bf16 q/k/v, fp32 lambda/beta, fp32 state and log)",
-            "config": config_of(wl, world), "roofline": res["roofline"],
+            "config": config_of(wl, world, a.tile_v), "roofline": res["roofline"],
             "gpu_launches": res["gpu_launches"],
             "hbm_tbs": res["roofline"]["achieved"] / 1e3}
     for k in ("eager", "deferred_bytes_per_step", "e2e", "clocks"):
