@@ -217,7 +217,7 @@ def run_gpu(a, wl, rank, world, dist):
 
     def flush_l2():
         flush.zero_()
-        torch.sum(flush_rd, out=flush_sink)
+        torch.sum(flush_rd, dim=0, out=flush_sink)
     L, K, W = wl.log_cap, a.steps, a.warmup
     ndist = max(1, min(wl.steps, 256 // wl.n_layers))
 
