@@ -8,15 +8,21 @@
 // heads (blockIdx.x, + gridDim.x, ...).
 //
 // Warp roles inside a CTA:
-//  * producer warp: reads the slot id and live-log length of the next heads,
-//    prefetches their live log entries and token rows into L2, and streams each
-//    head's base state in four contiguous 16 KB chunks (32 rows x 128 columns)
-//    into a ring of shared-memory stages with cp.async.bulk (TMA bulk copies,
-//    evict-first in L2), completing on per-stage mbarriers.
+//  * producer warp: prefetches the next heads' token rows into L2, reads their
+//    slot ids, and streams each head's base state in four contiguous 16 KB chunks
+//    (32 rows x 128 columns) into a ring of shared-memory stages with
+//    cp.async.bulk (TMA bulk copies, evict-first in L2), completing on per-stage
+//    mbarriers.  The copies go out as soon as the slot id is known; the live-log
+//    length, read meanwhile, is published with the stage's arrival (the phase
+//    completes only when both the bytes and the arrival are in), together with an
+//    L2 prefetch of the head's live log entries.
 //  * 8 consumer warps: token prescale and ReplayPrep coefficients, the two
 //    mat-vecs S^T qt and S^T kt over the staged chunks, the value-log replay,
 //    b_t and o_t, the log append -- or, on the slot's merge step, the write-back
 //    of the materialised state straight from the staged chunks.
+//  * finalizer warp: commits each slot's new live-log length (Finalize) with the
+//    arrival counters, so no consumer ever waits on a global atomic; consumers
+//    hand it (slot-layer, new length) through a small mbarrier-guarded ring.
 // Stages are released per chunk on append heads and after the write-back on
 // merge heads, so HBM streaming continues while consumers do the per-head work.
 //
@@ -39,7 +45,9 @@ constexpr int CFLOATS = CROWS * DV;              // floats per chunk
 constexpr uint32_t CBYTES = CFLOATS * 4;         // 16 KB
 constexpr int NCW = 8;                           // consumer warps
 constexpr int NCT = NCW * 32;                    // consumer threads
-constexpr int NTHREADS = NCT + 32;               // + producer warp
+constexpr int NTHREADS = NCT + 64;               // + producer warp + finalizer warp
+constexpr int PRODUCER = NCW, FINALIZER = NCW + 1;
+constexpr int NC = 8;                            // finalizer hand-off slots
 constexpr int RPW = CROWS / NCW;                 // rows per consumer warp per chunk
 constexpr int LMAX = 32;                         // log capacity supported here
 constexpr int EPW = LMAX / NCW;                  // log entries per warp in ReplayPrep
@@ -49,7 +57,7 @@ constexpr int BAR_CONS = 1;                      // named barrier of the consume
 
 // Byte offsets inside the dynamic shared-memory block.
 struct Layout {
-    size_t stages, A, b, red, vec, bt, cq, ck, idesc, flags, bars, total;
+    size_t stages, A, b, red, vec, bt, cq, ck, idesc, cinfo, flags, bars, total;
     __host__ __device__ Layout(int ns, int L) {
         const size_t L4 = (size_t)((L + 3) & ~3);
         size_t o = 0;
@@ -62,8 +70,9 @@ struct Layout {
         cq = o;     o += L4 * 4;
         ck = o;     o += L4 * 4;
         idesc = o;  o += (size_t)ns * 16;
+        cinfo = o;  o += (size_t)NC * 16;
         flags = o;  o += 16;
-        bars = o;   o += (size_t)2 * ns * 8;
+        bars = o;   o += (size_t)(2 * ns + 2 * NC) * 8;
         total = o;
     }
 };
@@ -91,8 +100,11 @@ __global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KPar
     int4 *idesc = reinterpret_cast<int4 *>(smem + lay.idesc);
     volatile int *flags = reinterpret_cast<volatile int *>(smem + lay.flags);
     float *s_kq = reinterpret_cast<float *>(smem + lay.flags) + 3;
+    int4 *cinfo = reinterpret_cast<int4 *>(smem + lay.cinfo);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
     uint64_t *empty = full + NS;
+    uint64_t *done = empty + NS;   // consumer -> finalizer: hand-off slot filled
+    uint64_t *cfree = done + NC;   // finalizer -> consumer: hand-off slot read
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_items = p.batch * p.H;
@@ -104,6 +116,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KPar
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], NCW);
         }
+        for (int s = 0; s < NC; ++s) {
+            ptx::mbar_init(&done[s], 1);
+            ptx::mbar_init(&cfree[s], 1);
+        }
         flags[0] = 0;  // abort
         flags[1] = 0;  // chunks issued
         flags[2] = 0;  // chunks waited by the consumers
@@ -111,77 +127,87 @@ __global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KPar
     }
     __syncthreads();
 
-    if (warp == NCW) {
+    if (warp == PRODUCER) {
         // ------------------------------------------------------------------ producer
         const uint64_t pol = ptx::policy_evict_first();
         int g = 0, n = 0;
         bool abort = false;
         for (int base = blockIdx.x; base < n_items && !abort; base += PB * G) {
             const int it = base + lane * G;
-            int s = -1, c = 0, st = 0;
+            int s = -1, c = 0, in_range = 0;
             if (lane < PB && it < n_items) {
                 const int bi = it / p.H, h = it % p.H;
+                // token rows depend on the batch row only: warm L2 first
+                const int gk = h / (p.H / p.Hk);
+                ptx::prefetch_l2_aligned(static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + gk) * DK,
+                                         DK * sizeof(IT));
+                ptx::prefetch_l2_aligned(static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + gk) * DK,
+                                         DK * sizeof(IT));
+                ptx::prefetch_l2_aligned(static_cast<const IT *>(p.v) + ((size_t)bi * p.H + h) * DV,
+                                         DV * sizeof(IT));
+                if (DECAY == DL_DECAY_DIAG && !p.lam_const)
+                    ptx::prefetch_l2_aligned(p.lam + ((size_t)bi * p.H + h) * DK, DK * 4);
                 s = p.slots[bi];
-                if (s < 0 || s >= p.n_slots) {
-                    st = DL_EBIT_SLOT_RANGE;
-                } else {
-                    const size_t sl = (size_t)s * p.n_layers + p.layer;
-                    c = p.log_len ? p.log_len[sl] : 0;
-                    if (p.eager) {
-                        if (c != 0) st = DL_EBIT_LIVE_LOG;
-                    } else if (c < 0 || c > p.L) {
-                        st = DL_EBIT_LOG_LEN;
-                    } else if (!(p.auto_merge && c >= p.L - 1) && c >= p.L) {
-                        st = DL_EBIT_LOG_FULL;
-                    }
-                }
-                if (st == 0) {  // warm L2 with what the consumers will read for this head
-                    const size_t head = ((size_t)s * p.n_layers + p.layer) * p.H + h;
-                    if (c > 0) ptx::prefetch_l2_aligned(p.log + head * (size_t)p.L * E, (uint32_t)(c * E * 4));
-                    const int gk = h / (p.H / p.Hk);
-                    const IT *qrow = static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + gk) * DK;
-                    const IT *krow = static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + gk) * DK;
-                    ptx::prefetch_l2_aligned(qrow, DK * sizeof(IT));
-                    ptx::prefetch_l2_aligned(krow, DK * sizeof(IT));
-                    ptx::prefetch_l2_aligned(static_cast<const IT *>(p.v) + ((size_t)bi * p.H + h) * DV,
-                                     DV * sizeof(IT));
-                    if (DECAY == DL_DECAY_DIAG && !p.lam_const)
-                        ptx::prefetch_l2_aligned(p.lam + ((size_t)bi * p.H + h) * DK, DK * 4);
-                }
+                in_range = (s >= 0 && s < p.n_slots);
+                // issued now, consumed when this head's stages are published
+                if (in_range && p.log_len) c = p.log_len[(size_t)s * p.n_layers + p.layer];
             }
             for (int k = 0; k < PB; ++k) {
                 const int itk = base + k * G;
                 if (itk >= n_items) break;
                 const int sk = __shfl_sync(0xffffffffu, s, k);
-                const int ck = __shfl_sync(0xffffffffu, c, k);
-                const int stk = __shfl_sync(0xffffffffu, st, k);
+                const int rk = __shfl_sync(0xffffffffu, in_range, k);
+                const int h = itk % p.H;
+                const size_t head = rk ? ((size_t)sk * p.n_layers + p.layer) * p.H + h : 0;
+                const int nch = rk ? NCHUNK : 1;
                 if (lane == 0) {
-                    if (stk) atomicOr(p.err, stk);
-                    const int bi = itk / p.H, h = itk % p.H;
-                    const size_t head = stk ? 0 : ((size_t)sk * p.n_layers + p.layer) * p.H + h;
                     const float *tile = p.state + head * (size_t)(DK * DV);
-                    const int merge_now = p.eager || (p.auto_merge && ck >= p.L - 1);
-                    const int nch = stk ? 1 : NCHUNK;
-                    (void)bi;
-                    for (int q = 0; q < nch; ++q, ++g) {
-                        const int sg = g % NS;
-                        if (!ptx::mbar_wait_bounded(&empty[sg], ((g / NS) & 1) ^ 1, WAIT_NS)) {
+                    int issued = 0;
+                    for (int q = 0; q < nch; ++q) {
+                        const int gq = g + q, sg = gq % NS;
+                        if (!ptx::mbar_wait_bounded(&empty[sg], ((gq / NS) & 1) ^ 1, WAIT_NS)) {
                             abort = true;
                             break;
                         }
-                        if (q == 0) idesc[n % NS] = make_int4(sk, ck, stk == 0, merge_now);
-                        if (stk) {
-                            ptx::mbar_arrive(&full[sg]);
-                        } else {
-                            ptx::mbar_arrive_expect_tx(&full[sg], CBYTES);
+                        if (rk) {
+                            ptx::mbar_expect_tx(&full[sg], CBYTES);
                             ptx::bulk_g2s(stages + (size_t)sg * CFLOATS, tile + (size_t)q * CFLOATS,
                                           CBYTES, &full[sg], pol);
+                            ++issued;
                         }
                     }
-                    ++n;
+                    if (abort && issued) {
+                        // publish the copies already in flight as a skipped head, so
+                        // their phases complete and the exit drain can wait for them
+                        idesc[n % NS] = make_int4(sk, 0, 4, 0);
+                        for (int q = 0; q < issued; ++q) ptx::mbar_arrive(&full[(g + q) % NS]);
+                        g += issued;
+                    }
                 }
                 abort = __shfl_sync(0xffffffffu, abort, 0);
                 if (abort) break;
+                // the live length decides the head's phase; publish it with the arrivals
+                const int ck = __shfl_sync(0xffffffffu, c, k);
+                if (lane == 0) {
+                    int st = rk ? 0 : DL_EBIT_SLOT_RANGE;
+                    if (rk) {
+                        if (p.eager) {
+                            if (ck != 0) st = DL_EBIT_LIVE_LOG;
+                        } else if (ck < 0 || ck > p.L) {
+                            st = DL_EBIT_LOG_LEN;
+                        } else if (!(p.auto_merge && ck >= p.L - 1) && ck >= p.L) {
+                            st = DL_EBIT_LOG_FULL;
+                        }
+                    }
+                    if (st) atomicOr(p.err, st);
+                    const int merge_now = p.eager || (p.auto_merge && ck >= p.L - 1);
+                    if (st == 0 && ck > 0)
+                        ptx::prefetch_l2_aligned(p.log + head * (size_t)p.L * E, (uint32_t)(ck * E * 4));
+                    idesc[n % NS] = make_int4(sk, ck, (st == 0 ? 1 : 0) | (merge_now ? 2 : 0) | (rk ? 4 : 0), 0);
+                    for (int q = 0; q < nch; ++q) ptx::mbar_arrive(&full[(g + q) % NS]);
+                    g += nch;
+                    ++n;
+                }
             }
         }
         if (lane == 0) {
@@ -191,29 +217,76 @@ __global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KPar
                 atomicOr(p.err, DL_EBIT_TIMEOUT);
             }
         }
+    } else if (warp == FINALIZER) {
+        // ------------------------------------------------------------------ finalizer
+        if (lane == 0 && !p.eager) {
+            bool abort = false;
+            int n = 0;
+            for (int it = blockIdx.x; it < n_items; it += G, ++n) {
+                const int cs = n % NC;
+                if (!ptx::mbar_wait_bounded(&done[cs], (n / NC) & 1, WAIT_NS)) {
+                    abort = true;
+                    break;
+                }
+                const int4 ci = cinfo[cs];
+                ptx::mbar_arrive(&cfree[cs]);
+                if (ci.z) {  // the last unit of a (slot, layer) commits its live length
+                    const int old = atomicAdd(p.arrive + ci.x, 1);
+                    if (old == p.H - 1) {
+                        p.log_len[ci.x] = ci.y;
+                        p.arrive[ci.x] = 0;
+                    }
+                }
+            }
+            if (abort) {
+                flags[0] = 1;
+                atomicOr(p.err, DL_EBIT_TIMEOUT);
+            }
+        }
     } else {
         // ------------------------------------------------------------------ consumers
         const int t = tid;
         int g = 0, gw = 0, n = 0;
-        bool abort = false;
+        bool abort = false, handoff_late = false;
+        // hand (slot-layer, new live length) of head n to the finalizer warp
+        auto hand_off = [&](int n_, int sl_, int len_, int commit_) {
+            if (t != 0 || p.eager) return;
+            const int cs = n_ % NC;
+            if (!ptx::mbar_wait_bounded(&cfree[cs], ((n_ / NC) & 1) ^ 1, WAIT_NS)) {
+                handoff_late = true;
+                return;
+            }
+            cinfo[cs] = make_int4(sl_, len_, commit_, 0);
+            ptx::mbar_arrive(&done[cs]);
+        };
         for (int it = blockIdx.x; it < n_items; it += G, ++n) {
             {
                 const bool ok = ptx::mbar_wait_bounded(&full[g % NS], (g / NS) & 1, WAIT_NS);
-                if (ptx::bar_or(BAR_CONS, NCT, !ok)) {
+                if (ptx::bar_or(BAR_CONS, NCT, !ok || handoff_late)) {
                     abort = true;
                     break;
                 }
                 ++gw;
             }
             const int4 d = idesc[n % NS];
-            if (!d.z) {  // skipped head: one empty stage was sent
+            if (!(d.z & 1)) {  // skipped head: drain the stages it was sent, then release them
+                const int nch = (d.z & 4) ? NCHUNK : 1;
+                for (int q = 1; q < nch && !abort; ++q) {
+                    const int gq = g + q;
+                    const bool ok = ptx::mbar_wait_bounded(&full[gq % NS], (gq / NS) & 1, WAIT_NS);
+                    if (ptx::bar_or(BAR_CONS, NCT, !ok)) abort = true;
+                    else ++gw;
+                }
+                if (abort) break;
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&empty[g % NS]);
-                ++g;
+                if (lane == 0)
+                    for (int q = 0; q < nch; ++q) ptx::mbar_arrive(&empty[(g + q) % NS]);
+                g += nch;
+                hand_off(n, 0, 0, 0);
                 continue;
             }
             const int s = d.x, c = d.y;
-            const bool merge_now = d.w != 0;
+            const bool merge_now = (d.z & 2) != 0;
             const int bi = it / p.H, h = it % p.H;
             const size_t sl = (size_t)s * p.n_layers + p.layer;
             const size_t head = sl * p.H + h;
@@ -415,21 +488,14 @@ __global__ void __launch_bounds__(NTHREADS, 2) persistent_step_kernel(const KPar
             }
             g += NCHUNK;
 
-            // -- Finalize: after every consumer is done with this head, the last unit
-            //    of the (slot, layer) commits the live length
+            // -- Finalize: once every consumer is done with this head, hand the new
+            //    live length to the finalizer warp (which commits it for the slot)
             ptx::bar_sync(BAR_CONS, NCT);
-            if (t == 0 && !p.eager) {
-                __threadfence();
-                const int old = atomicAdd(p.arrive + sl, 1);
-                if (old == p.H - 1) {
-                    p.log_len[sl] = merge_now ? 0 : c + 1;
-                    p.arrive[sl] = 0;
-                }
-            }
+            hand_off(n, (int)sl, merge_now ? 0 : c + 1, 1);
         }
         if (t == 0) {
             flags[2] = gw;
-            if (abort) {
+            if (abort || handoff_late) {
                 flags[0] = 1;
                 atomicOr(p.err, DL_EBIT_TIMEOUT);
             }
