@@ -203,6 +203,39 @@ dl_status dl_materialize(dl_pool *pool, int32_t layer, const int32_t *slots, int
  * `clear` is non-zero.  Returns DL_ERR_DEVICE when any bit was set. */
 dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *stream);
 
+/* Decode step that allocates nothing.  The paper has no counterpart: this entry
+ * point exists for integration only.
+ *
+ * Who needs it.  dl_decode_step needs one small buffer besides the state, the
+ * log and the step's inputs and outputs: the per-(slot, layer) arrival counters
+ * (pool `arrive`) that let the last work unit of a slot commit its new live-log
+ * length.  Some callers cannot provide even that.  One example is a serving engine
+ * whose memory manager has already divided the whole device among its own pools
+ * and refuses further cudaMalloc calls.  Another is a host runtime that reaches the
+ * GPU only through buffers it was handed at start-up.  This call keeps the
+ * counters in a fixed array compiled into the library instead, so such a caller
+ * passes only memory it already owns.
+ *
+ * Arguments and results are those of dl_decode_step, except that the pool is a
+ * descriptor (checked on every call with the rules of dl_create_pool; no handle
+ * is made) and its `arrive` field is ignored and may be NULL.  The descriptor must
+ * name a log.
+ *
+ * Limits and sharing:
+ *  - n_slots * n_layers <= DL_NOALLOC_MAX_COUNTERS, else DL_ERR_SHAPE.  The array
+ *    (DL_NOALLOC_MAX_COUNTERS int32, 256 KiB) occupies every GPU that loads the
+ *    library until the process exits.
+ *  - All calls share that one array.  Each call first clears the counters it uses
+ *    (an asynchronous memset on `stream`), so calls that overlap on the GPU (two
+ *    streams, or two host threads) race; issue them in order on one stream.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, which can load the module).  Make that first call
+ *    before any stream capture.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine. */
+#define DL_NOALLOC_MAX_COUNTERS 65536
+dl_status dl_decode_step_noalloc(const dl_pool_desc *desc, int32_t layer,
+                                 const dl_step_args *args, int32_t auto_merge, void *stream);
+
 /* Static description of a status code. */
 const char *dl_status_string(dl_status status);
 

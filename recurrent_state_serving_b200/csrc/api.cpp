@@ -240,3 +240,41 @@ DL_API const char *dl_status_string(dl_status status) {
     }
     return "unknown status";
 }
+
+namespace dl {
+
+// Checks a bare descriptor with the rules of dl_create_pool, except that its
+// arrival-counter buffer is not looked at (the entry point that allocates nothing
+// supplies its own).  Makes no CUDA call.
+dl_status check_desc_without_arrive(const dl_pool_desc &d) {
+    if (d.n_slots <= 0 || d.n_layers <= 0 || d.n_heads <= 0 || d.n_kheads <= 0)
+        return DL_ERR_SHAPE;
+    if (d.n_heads % d.n_kheads) return DL_ERR_SHAPE;
+    if (!dk_supported(d.d_k)) return DL_ERR_SHAPE;
+    if (d.d_v < 16 || d.d_v > 1024 || d.d_v % 16) return DL_ERR_SHAPE;
+    if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
+    if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32 && d.tile_v != 128) return DL_ERR_SHAPE;
+    if (d.tile_v == 32 && (d.d_k < 64 || d.d_v % 32)) return DL_ERR_SHAPE;
+    if (d.tile_v == 128 && !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return DL_ERR_SHAPE;
+    if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
+    if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
+        return DL_ERR_INVALID_ARG;
+    if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
+        return DL_ERR_INVALID_ARG;
+    if (!d.log || !aligned(d.log, 16) || !d.log_len || !aligned(d.log_len, 4))
+        return DL_ERR_INVALID_ARG;
+    if ((long long)d.n_slots * d.n_heads * (d.d_v / 16) > 0x7fffffffLL) return DL_ERR_SHAPE;
+    return DL_OK;
+}
+
+// Runs dl_decode_step for a checked descriptor with the given arrival counters,
+// through a pool handle held on the stack (nothing is allocated).
+dl_status decode_step_on_desc(const dl_pool_desc &desc, int32_t *arrive, int32_t layer,
+                              const dl_step_args *args, int32_t auto_merge, void *stream) {
+    dl_pool stack_pool;
+    stack_pool.d = desc;
+    stack_pool.d.arrive = arrive;
+    return dl_decode_step(&stack_pool, layer, args, auto_merge, stream);
+}
+
+}  // namespace dl

@@ -61,10 +61,12 @@ _lib.dl_merge.argtypes = [_vp, ctypes.c_int32, _vp, ctypes.c_int32, _vp]
 _lib.dl_materialize.argtypes = [_vp, ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp]
 _lib.dl_reset_slots.argtypes = [_vp, _vp, ctypes.c_int32, _vp]
 _lib.dl_read_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, _vp]
+_lib.dl_decode_step_noalloc.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.c_int32,
+                                        ctypes.POINTER(dl_step_args), ctypes.c_int32, _vp]
 _lib.dl_status_string.argtypes = [ctypes.c_int]
 _lib.dl_status_string.restype = ctypes.c_char_p
 for _f in ("dl_create_pool", "dl_destroy_pool", "dl_decode_step", "dl_append", "dl_eager_step",
-           "dl_merge", "dl_materialize", "dl_reset_slots", "dl_read_error"):
+           "dl_merge", "dl_materialize", "dl_reset_slots", "dl_read_error", "dl_decode_step_noalloc"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -192,6 +194,25 @@ def dl_decode_step(pool: Pool, layer: int, slots, q, k, v, lam=None, beta=None, 
     a = _step_args(pool, slots, q, k, v, lam, beta, out, lambda_per_head)
     _check(_lib.dl_decode_step(pool.handle, layer, ctypes.byref(a), 1 if auto_merge else 0,
                                _stream(stream)), "dl_decode_step")
+    return out
+
+
+def dl_decode_step_noalloc(pool: Pool, layer: int, slots, q, k, v, lam=None, beta=None, out=None,
+                           lambda_per_head=False, auto_merge=True, stream=None):
+    """dl_decode_step without the caller's arrival-counter buffer: the library keeps
+    the counters in a fixed device array of its own (for callers that cannot
+    allocate device memory).  The pool's descriptor is passed with `arrive` unset;
+    the pool's own `arrive` tensor is not touched.  Calls must not overlap on the
+    GPU (they share the array)."""
+    if out is None:
+        out = torch.empty(slots.numel(), pool.n_heads, pool.d_v, dtype=torch.float32,
+                          device=pool.state.device)
+    a = _step_args(pool, slots, q, k, v, lam, beta, out, lambda_per_head)
+    desc = dl_pool_desc.from_buffer_copy(pool.desc)
+    desc.arrive = None
+    _check(_lib.dl_decode_step_noalloc(ctypes.byref(desc), layer, ctypes.byref(a),
+                                       1 if auto_merge else 0, _stream(stream)),
+           "dl_decode_step_noalloc")
     return out
 
 

@@ -8,9 +8,9 @@ import pytest
 
 from recurrent_state_serving_b200 import deltalog as dl
 
-EXPECTED = ["dl_append", "dl_create_pool", "dl_decode_step", "dl_destroy_pool",
-            "dl_eager_step", "dl_materialize", "dl_merge", "dl_read_error", "dl_reset_slots",
-            "dl_status_string"]
+EXPECTED = ["dl_append", "dl_create_pool", "dl_decode_step", "dl_decode_step_noalloc",
+            "dl_destroy_pool", "dl_eager_step", "dl_materialize", "dl_merge", "dl_read_error",
+            "dl_reset_slots", "dl_status_string"]
 
 
 def test_header_declares_the_boundary():
@@ -147,3 +147,24 @@ def test_status_strings():
     for s in range(7):
         assert dl.dl_status_string(s) and dl.dl_status_string(s) != "unknown status"
     assert dl.dl_status_string(99) == "unknown status"
+
+
+def test_noalloc_entry_point_checks_without_gpu():
+    """The allocation-free decode step validates its descriptor on the host (with the
+    rules of dl_create_pool, minus the arrival buffer) before any CUDA call."""
+    lib = dl.library()
+    P = 0x60000
+    a = dl.dl_step_args(P, 0, P, P, P, 1, P, 0, P, P)   # empty batch: no launch
+
+    def call(**kw):
+        d = _desc(**kw)
+        return lib.dl_decode_step_noalloc(ctypes.byref(d), 0, ctypes.byref(a), 1, None)
+
+    assert call(arrive=None) == dl.DL_OK
+    assert call() == dl.DL_OK                           # a given arrive buffer is ignored
+    assert call(arrive=None, log=None) == dl.DL_ERR_INVALID_ARG
+    assert call(arrive=None, log_len=None) == dl.DL_ERR_INVALID_ARG
+    assert call(arrive=None, d_k=100) == dl.DL_ERR_SHAPE
+    assert call(arrive=None, n_slots=65536, n_layers=2) == dl.DL_ERR_SHAPE   # > 65536 counters
+    assert call(arrive=None, n_slots=32768, n_layers=2) == dl.DL_OK
+    assert lib.dl_decode_step_noalloc(None, 0, ctypes.byref(a), 1, None) == dl.DL_ERR_INVALID_ARG
