@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--traffic-from", default=None,
+                    help="write profiles/step_kernel_traffic.txt from an ncu csv and exit")
     ap.add_argument("--tile-v", type=int, default=0,
                     help="work-unit width: 0 automatic, 16/32 value tiles, 128 whole heads")
     return ap.parse_args()
@@ -86,6 +88,40 @@ def config_of(wl, n_gpus, tile_v=0):
             "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
             "l2": "flushed before every timed step, outside the timed interval: 256 MiB write, then 256 MiB read of another buffer (evicts the dirty lines)",
             "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
+
+
+def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str) -> str:
+    """Text for profiles/step_kernel_traffic.txt from an ncu --csv export of
+    dram__bytes_read.sum and dram__bytes_write.sum over consecutive launches of the
+    hot kernel (one full merge interval, so the mix of append and merge launches
+    matches the timed region).  Run: python bench.py --traffic-from <csv>."""
+    import csv
+    import re
+    rows = list(csv.reader(open(csv_path)))
+    i = [k for k, r in enumerate(rows) if "Kernel Name" in r][0]
+    hdr = rows[i]
+    kn, mn, mv = hdr.index("Kernel Name"), hdr.index("Metric Name"), hdr.index("Metric Value")
+    mu = hdr.index("Metric Unit") if "Metric Unit" in hdr else None
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    per = {}
+    idcol = hdr.index("ID") if "ID" in hdr else None
+    for r in rows[i + 1:]:
+        if len(r) <= mv or not re.search(kernel_regex, r[kn]):
+            continue
+        if r[mn] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        v = float(r[mv].replace(",", "")) * scale.get(r[mu] if mu is not None else "byte", 1)
+        key = r[idcol] if idcol is not None else len(per)
+        per[key] = per.get(key, 0.0) + v
+    vals = list(per.values())
+    if not vals:
+        raise SystemExit("no matching launches in " + csv_path)
+    avg = sum(vals) / len(vals)
+    return (f"# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the hot kernel,\n"
+            f"# averaged over {len(vals)} consecutive launches (one merge interval).\n"
+            f"workload = {workload_key}\nkernel_sha = {kernel_source_hash()}\n"
+            f"launches = {len(vals)}\ndram_bytes_per_launch = {avg:.0f}\n"
+            f"min_launch_bytes = {min(vals):.0f}\nmax_launch_bytes = {max(vals):.0f}\n")
 
 
 def measured_peaks():
@@ -181,9 +217,9 @@ class ClockSampler:
 # ranks
 # ---------------------------------------------------------------------------------
 def res_kernel_name(wl, tile_v):
-    whole = tile_v == 128 or (tile_v == 0 and wl.d_k == 128 and wl.d_v == 128 and wl.log_cap <= 32
-                              and wl.batch * wl.n_heads >= 2 * 148)
-    return "dl::pk::persistent_step_kernel" if whole else "dl::step_kernel"
+    whole = tile_v == 128 or (tile_v == 0 and wl.d_k == 128 and wl.d_v == 128
+                              and wl.batch * wl.n_heads >= 148)
+    return "dl::wh::warp_head_kernel" if whole else "dl::step_kernel"
 
 
 def max_over_ranks(x: float, dist=None, device=None) -> float:
@@ -361,38 +397,40 @@ def run_gpu(a, wl, rank, world, dist):
 # ---------------------------------------------------------------------------------
 def oracle_sample_rate(wl, target_s=10.0):
     """fp64 eager oracle on the host cores over a bounded sample of the workload's
-    heads (layer 0); returns (head-steps/s, threads, description)."""
+    heads (layer 0); returns (head-steps/s, threads, description).  Up to 64
+    distinct seeded steps are generated and cycled to reach about target_s of
+    oracle work; only the oracle call is timed."""
     import oracle
     from recurrent_state_serving_b200 import synth
     threads = os.cpu_count() or 1
-    x = synth.step_inputs(wl, 0, 0)
     S0 = synth.initial_state(wl.with_(batch=min(wl.batch, 64)), 0).astype(np.float64)
     rows = np.arange(S0.shape[0])
+    ndist = min(64, wl.steps)
+    seq = [synth.select_rows(wl, synth.step_inputs(wl, t, 0), rows) for t in range(ndist)]
+    f = lambda k, t: synth.input_to_f64(seq[t % ndist][k], wl.in_dtype)
 
     def run(T):
-        seq = [synth.select_rows(wl, synth.step_inputs(wl, t, 0), rows) for t in range(T)]
-        f = lambda k, t: synth.input_to_f64(seq[t][k], wl.in_dtype)
         Q = np.stack([f("q", t) for t in range(T)])
         Kk = np.stack([f("k", t) for t in range(T)])
         V = np.stack([f("v", t) for t in range(T)])
         LAM = None
         if wl.decay != "none":
             LAM = seq[0]["lam"].astype(np.float64) if wl.lambda_const else np.stack(
-                [seq[t]["lam"].astype(np.float64) for t in range(T)])
-        BETA = np.stack([seq[t]["beta"].astype(np.float64) for t in range(T)]) if wl.update == "delta" else None
+                [seq[t % ndist]["lam"].astype(np.float64) for t in range(T)])
+        BETA = (np.stack([seq[t % ndist]["beta"].astype(np.float64) for t in range(T)])
+                if wl.update == "delta" else None)
         t0 = time.perf_counter()
         oracle.eager_rollout(S0, Q, Kk, V, LAM, BETA, decay=wl.decay, update=wl.update,
                              lambda_const=wl.lambda_const, threads=threads)
         return time.perf_counter() - t0
 
-    dt = run(2)
+    dt = run(8)
     heads = S0.shape[0] * wl.n_heads
-    per_step = dt / 2
-    T = int(max(2, min(512, target_s / max(per_step, 1e-6))))
+    T = int(max(8, min(4096, 8 * target_s / max(dt, 1e-6))))
     dt = run(T)
     rate = heads * T / dt
     desc = (f"{heads} heads ({S0.shape[0]} slots x {wl.n_heads} heads, layer 0) x {T} steps of "
-            f"{wl.name}, fp64 eager oracle, {dt:.1f} s")
+            f"{wl.name} ({ndist} distinct seeded steps cycled), fp64 eager oracle, {dt:.1f} s")
     return rate, threads, desc
 
 
@@ -442,6 +480,12 @@ def main():
     a = parse()
     sys.path.insert(0, ROOT)
     wl = workload(a)
+    if a.traffic_from:
+        key = config_of(wl, 1)["workload"]
+        text = traffic_summary_from_ncu(a.traffic_from, key, r"warp_head_kernel|step_kernel")
+        open(PROFILE_TRAFFIC, "w").write(text)
+        print(text)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
 

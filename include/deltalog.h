@@ -106,12 +106,14 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
  *           them to zero at the end of every call.  Required with a log.
  *  err_word [1] int32 sticky device error bits; zero it before first use.
  *  tile_v   value-tile width B_V of a work unit (Section 3.3): 16 or 32 columns;
- *           128 for whole-head work units run by the persistent, TMA-staged decode
- *           kernel (needs d_k = d_v = 128 and log_cap <= 32; other calls of such a
- *           pool use 16/32-wide tiles); 0 to choose per launch (whole heads for
- *           d_k = d_v = 128, log_cap <= 32 and at least two heads per CTA slot,
- *           else 32 columns unless that leaves SMs idle, else 16).  32 needs
- *           d_k >= 64 and d_v a multiple of 32.
+ *           128 for whole-head work units, each owned by one warp of the
+ *           warp-per-head decode kernel (needs d_k = d_v = 128; it serves decode
+ *           and eager steps whose q, k, v, per-key lambda and out are 16-byte
+ *           aligned, and other calls of such a pool use 16/32-wide tiles); 0 to
+ *           choose per launch (whole heads for decode steps when those conditions
+ *           hold and there are at least as many heads as SMs, else 32 columns
+ *           unless that leaves SMs idle, else 16).  32 needs d_k >= 64 and d_v a
+ *           multiple of 32.
  *
  * The cumulative log-decay lbar of a slot is not stored separately: it equals
  * Lambda of the newest live entry (0 when the log is empty).

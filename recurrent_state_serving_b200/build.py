@@ -31,7 +31,7 @@ STEP_DKS = (16, 64, 128)
 def _sources():
     units = [("api", os.path.join(CSRC, "api.cpp"), []),
              ("kernels_merge", os.path.join(CSRC, "kernels_merge.cu"), []),
-             ("kernels_persistent", os.path.join(CSRC, "kernels_persistent.cu"), []),
+             ("kernels_warp_head", os.path.join(CSRC, "kernels_warp_head.cu"), []),
              ("noalloc", os.path.join(CSRC, "noalloc.cu"), [])]
     for dk in STEP_DKS:
         units.append((f"kernels_step_dk{dk}", os.path.join(CSRC, "kernels_step.cu"),

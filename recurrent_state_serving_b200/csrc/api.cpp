@@ -48,12 +48,21 @@ void set_tiles(const dl_pool_desc &d, dl::KParams &p, int batch, int &bv) {
     p.nv = p.dv / bv;
 }
 
-// Full-head work units (persistent kernel) for a decode or eager step?
-bool use_persistent(const dl_pool_desc &d, int batch, bool want_out) {
-    if (!want_out || !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return false;
+// Whole-head work units (warp-per-head kernel) for a decode or eager step?  That
+// kernel streams token rows and writes outputs with 128-bit accesses, so it needs
+// 16-byte aligned q, k, v, per-key lambda and out; calls whose buffers are only
+// element-aligned run the value-tiled kernel.
+bool use_whole_head(const dl_pool_desc &d, const dl_step_args *a, bool want_out, bool eager) {
+    if (!want_out || !dl::whole_head_supported(d.d_k, d.d_v)) return false;
+    if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->out, 16))
+        return false;
+    if (d.decay == DL_DECAY_DIAG && !aligned(a->lambda, 16)) return false;
     if (d.tile_v == 128) return true;
     if (d.tile_v != 0) return false;
-    return (long long)batch * d.n_heads >= 2LL * dl::device_sm_count();
+    // An eager step rewrites the whole state: the value-tiled kernel, which keeps
+    // its tile in registers between the read and the write, measured faster.
+    if (eager) return false;
+    return (long long)a->batch * d.n_heads >= (long long)dl::device_sm_count();
 }
 
 dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, bool need_out) {
@@ -93,9 +102,9 @@ dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_o
     p.want_out = want_out ? 1 : 0;
     p.undecayed = d.update == DL_UPDATE_DELTA_UNDECAYED ? 1 : 0;
     cudaError_t e;
-    if (use_persistent(d, a->batch, want_out)) {
+    if (use_whole_head(d, a, want_out, eager)) {
         p.nv = 1;
-        e = dl::launch_persistent(p, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
+        e = dl::launch_whole_head(p, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
                                   static_cast<cudaStream_t>(stream));
     } else {
         int bv = 32;
@@ -120,7 +129,7 @@ DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
     if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
     if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32 && d.tile_v != 128) return DL_ERR_SHAPE;
     if (d.tile_v == 32 && (d.d_k < 64 || d.d_v % 32)) return DL_ERR_SHAPE;
-    if (d.tile_v == 128 && !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return DL_ERR_SHAPE;
+    if (d.tile_v == 128 && !dl::whole_head_supported(d.d_k, d.d_v)) return DL_ERR_SHAPE;
     if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;
@@ -255,7 +264,7 @@ dl_status check_desc_without_arrive(const dl_pool_desc &d) {
     if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
     if (d.tile_v != 0 && d.tile_v != 16 && d.tile_v != 32 && d.tile_v != 128) return DL_ERR_SHAPE;
     if (d.tile_v == 32 && (d.d_k < 64 || d.d_v % 32)) return DL_ERR_SHAPE;
-    if (d.tile_v == 128 && !dl::persistent_supported(d.d_k, d.d_v, d.log_cap)) return DL_ERR_SHAPE;
+    if (d.tile_v == 128 && !dl::whole_head_supported(d.d_k, d.d_v)) return DL_ERR_SHAPE;
     if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;

@@ -36,7 +36,6 @@ struct KParams {
     int eager;       // eager step: c = 0 and always write back, no log
     int want_out;    // write o_t
     int undecayed;   // delta correction from S_{t-1} instead of Diag(e^lambda) S_{t-1}
-    int ns;          // shared-memory stages of the persistent kernel (set by its launcher)
 };
 
 // Value-tile width chosen for a launch (16 or 32 columns).
@@ -44,10 +43,10 @@ int pick_bv(int dk, int dv, long long work_items_at_32);
 
 cudaError_t launch_step(const KParams &p, int bv, int decay, bool delta, bool bf16,
                         cudaStream_t st);
-// Persistent TMA-staged step for full 128 x 128 heads (dl_persistent.cuh).
-bool persistent_supported(int dk, int dv, int log_cap);
+// Warp-per-head step for full 128 x 128 heads (dl_warp_head.cuh).
+bool whole_head_supported(int dk, int dv);
 int device_sm_count();
-cudaError_t launch_persistent(const KParams &p, int decay, bool delta, bool bf16, cudaStream_t st);
+cudaError_t launch_whole_head(const KParams &p, int decay, bool delta, bool bf16, cudaStream_t st);
 
 cudaError_t launch_merge(const KParams &p, int bv, int decay, bool materialize,
                          cudaStream_t st);

@@ -70,6 +70,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return true;
 }
 
+// Order this thread's prior generic-proxy accesses to shared memory before later
+// async-proxy (bulk copy) accesses, e.g. before a stage that was just read is
+// refilled by cp.async.bulk.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's prior generic-proxy writes to global memory before later
+// async-proxy reads of it (a bulk copy re-reading data the thread just wrote).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// L2 policy: keep the line (data read again soon).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // L2 policy: evict the line first (data streamed once).
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t pol;

@@ -1,5 +1,5 @@
-// Launch of the persistent TMA-staged decode step (dl_persistent.cuh).
-#include "dl_persistent.cuh"
+// Launch of the warp-per-head decode step (dl_warp_head.cuh).
+#include "dl_warp_head.cuh"
 
 namespace dl {
 
@@ -16,34 +16,24 @@ int device_sm_count() {
     return cached[dev];
 }
 
-bool persistent_supported(int dk, int dv, int log_cap) {
-    return dk == pk::DK && dv == pk::DV && log_cap <= pk::LMAX;
-}
+bool whole_head_supported(int dk, int dv) { return dk == wh::DK && dv == wh::DV; }
 
 namespace {
 
-// Shared memory for two CTAs per SM: 228 KB per SM less 1 KB reserved per CTA.
-constexpr size_t kSmemPerCta = 115712;
-
 template <int DECAY, bool DELTA, typename IT>
-cudaError_t launch_one(KParams p, cudaStream_t st) {
-    auto kern = pk::persistent_step_kernel<DECAY, DELTA, IT>;
-    const size_t fixed = pk::Layout(0, p.L).total;
-    int ns = (int)((kSmemPerCta - fixed) / pk::CBYTES);
-    ns = ns < pk::NCHUNK ? pk::NCHUNK : (ns > 8 ? 8 : ns);
-    p.ns = ns;
-    const size_t smem = pk::Layout(ns, p.L).total;
-    static size_t configured = 0;  // per instantiation
-    if (smem > configured) {
+cudaError_t launch_one(const KParams &p, cudaStream_t st) {
+    auto kern = wh::warp_head_kernel<DECAY, DELTA, IT>;
+    static bool configured = false;  // per instantiation
+    if (!configured) {
         const cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wh::SMEM);
         if (e != cudaSuccess) return e;
-        configured = smem;
+        configured = true;
     }
     const long long items = (long long)p.batch * p.H;
-    const long long cap = 2LL * device_sm_count();
-    const int grid = (int)(items < cap ? items : cap);
-    kern<<<grid, pk::NTHREADS, smem, st>>>(p);
+    const long long sms = device_sm_count();
+    const int grid = (int)(items < sms ? items : sms);
+    kern<<<grid, wh::NTHREADS, wh::SMEM, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -58,7 +48,7 @@ cudaError_t by_update(const KParams &p, bool delta, bool bf16, cudaStream_t st) 
 
 }  // namespace
 
-cudaError_t launch_persistent(const KParams &p, int decay, bool delta, bool bf16, cudaStream_t st) {
+cudaError_t launch_whole_head(const KParams &p, int decay, bool delta, bool bf16, cudaStream_t st) {
     switch (decay) {
     case DL_DECAY_NONE: return by_update<DL_DECAY_NONE>(p, delta, bf16, st);
     case DL_DECAY_SCALAR: return by_update<DL_DECAY_SCALAR>(p, delta, bf16, st);

@@ -49,7 +49,7 @@ def test_create_pool_accepts_valid_descriptors():
     for kw in ({}, dict(d_k=16, d_v=16, n_kheads=4), dict(d_k=64, d_v=80), dict(log_cap=1),
                dict(log_cap=64), dict(log=None, log_len=None, arrive=None), dict(decay=0, update=0),
                dict(tile_v=16), dict(tile_v=32), dict(d_k=64, d_v=96, tile_v=32),
-               dict(tile_v=128, log_cap=32)):
+               dict(tile_v=128, log_cap=32), dict(tile_v=128, log_cap=64)):
         st, h = _create(_desc(**kw))
         assert st == dl.DL_OK, (kw, dl.dl_status_string(st))
         assert dl.library().dl_destroy_pool(h) == dl.DL_OK
@@ -75,7 +75,6 @@ def test_create_pool_accepts_valid_descriptors():
     (dict(tile_v=8), dl.DL_ERR_SHAPE),
     (dict(tile_v=32, d_k=16, d_v=32), dl.DL_ERR_SHAPE),
     (dict(tile_v=32, d_v=80), dl.DL_ERR_SHAPE),
-    (dict(tile_v=128, log_cap=33), dl.DL_ERR_SHAPE),
     (dict(tile_v=128, d_k=64, d_v=128), dl.DL_ERR_SHAPE),
     (dict(tile_v=128, d_v=256), dl.DL_ERR_SHAPE),
     (dict(tile_v=64), dl.DL_ERR_SHAPE),
