@@ -7,11 +7,21 @@
 A step is one decode step of the whole batch over all layers of the workload (one
 library call per layer), with every slot advancing by one token; merges happen on
 each slot's own merge step inside the same call.  Inputs are seeded synthetic
-tensors resident in HBM before timing starts.  Before every timed step, outside the
-timed interval, L2 (126 MB) is flushed by writing a 256 MiB buffer and then reading
-a second 256 MiB buffer: the read evicts the dirty lines the write left, so their
-write-back is not charged to the timed kernel and it starts from a cold, clean L2.
-Each step is bracketed by CUDA events on the launching stream.
+tensors resident in HBM before timing starts.
+
+Cold L2 between steps, two ways (``--l2``):
+  rotate (default)  inputs larger than L2: the pool holds R disjoint copies of the
+                    batch's slots, stepped in turn (step j uses group j mod R), with R
+                    the smallest count whose base states total >= 384 MiB (three times
+                    the 126 MB L2); R = 1 when one step's state is that large already.
+                    A step's state was last touched >= 2 L2-sizes of traffic earlier.
+                    The K steps run back to back between one pair of CUDA events,
+                    launched from a CUDA graph (``--launch graph``, default) or
+                    directly (``--launch stream``).
+  flush             before every timed step, outside the timed interval, L2 is
+                    flushed by writing a 256 MiB buffer and then reading a second
+                    256 MiB buffer (the read evicts the dirty lines the write left);
+                    each step is bracketed by its own CUDA events.
 
 Multi-GPU (torchrun, one process per GPU): the slots are independent, so each rank
 runs its own replica of the workload (weak scaling, no collective on the data
@@ -38,6 +48,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "decode head-steps/s (batch x heads x layers)"
 UNIT = "head-steps/s"
 FLUSH_BYTES = 256 << 20
+ROTATE_MIN_BYTES = 384 << 20  # base-state bytes of one rotation: three times L2 (126 MB)
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "step_kernel_traffic.txt")
 CSRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc")
 
@@ -67,6 +78,10 @@ def parse():
                     help="write profiles/step_kernel_traffic.txt from an ncu csv and exit")
     ap.add_argument("--tile-v", type=int, default=0,
                     help="work-unit width: 0 automatic, 16/32 value tiles, 128 whole heads")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                    help="cold L2 per step: rotate slot groups (inputs > L2) or flush before each step")
+    ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
+                    help="rotate mode: replay the timed steps from a CUDA graph or launch them directly")
     return ap.parse_args()
 
 
@@ -80,13 +95,33 @@ def workload(a):
     return wl
 
 
-def config_of(wl, n_gpus, tile_v=0):
+def rotation_groups(wl, l2_mode: str) -> int:
+    """Slot groups stepped in turn so that the base states of one rotation total at
+    least ROTATE_MIN_BYTES (1 under the flush method, or when one step's are enough)."""
+    if l2_mode == "flush":
+        return 1
+    step_state = wl.units_per_step * 4 * wl.d_k * wl.d_v
+    return max(1, -(-ROTATE_MIN_BYTES // step_state))
+
+
+def l2_description(wl, l2_mode: str, launch: str) -> str:
+    if l2_mode == "flush":
+        return ("flushed before every timed step, outside the timed interval: 256 MiB write, then "
+                "256 MiB read of another buffer (evicts the dirty lines); per-step CUDA events")
+    R = rotation_groups(wl, l2_mode)
+    mib = R * wl.units_per_step * 4 * wl.d_k * wl.d_v / 2**20
+    return (f"inputs larger than L2: {R} slot group(s) of the batch stepped in turn, {mib:.0f} MiB of "
+            f"base state per rotation (L2 126 MB); timed steps back to back, "
+            f"{'replayed from one CUDA graph' if launch == 'graph' else 'launched directly'}")
+
+
+def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph"):
     return {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}",
             "tile_v": tile_v or "auto",
             "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
             "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
             "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
-            "l2": "flushed before every timed step, outside the timed interval: 256 MiB write, then 256 MiB read of another buffer (evicts the dirty lines)",
+            "l2": l2_description(wl, l2_mode, launch),
             "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
 
 
@@ -237,6 +272,30 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms / 1e3)
 
 
+def live_entries(offsets, step_index: int, n_groups: int, log_cap: int):
+    """Live log entries each slot of the group stepped at global step ``step_index``
+    holds when the step starts: that group has taken step_index // n_groups steps
+    before it, after its staggering pre-steps."""
+    return (offsets + step_index // n_groups) % log_cap
+
+
+def graph_upload(graph, stream) -> bool:
+    """Upload an instantiated CUDA graph to the device ahead of its first replay, so
+    the replay inside the timed interval carries no upload work."""
+    import ctypes
+    try:
+        rt = ctypes.CDLL("libcudart.so.12")
+        ex = graph.raw_cuda_graph_exec()
+        if not isinstance(ex, int):
+            get = ctypes.pythonapi.PyCapsule_GetPointer
+            get.restype, get.argtypes = ctypes.c_void_p, [ctypes.py_object, ctypes.c_char_p]
+            ex = get(ex, None)
+        rt.cudaGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        return rt.cudaGraphUpload(ctypes.c_void_p(ex), ctypes.c_void_p(stream.cuda_stream)) == 0
+    except (OSError, AttributeError, TypeError, ValueError):
+        return False
+
+
 # ---------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------
@@ -247,9 +306,10 @@ def run_gpu(a, wl, rank, world, dist):
     from recurrent_state_serving_b200.runner import DecodeRunner
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    if a.l2 == "flush":
+        flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def flush_l2():
         flush.zero_()
@@ -270,56 +330,98 @@ def run_gpu(a, wl, rank, world, dist):
     sampler = ClockSampler(dev.index)
     sampler.start()
 
-    def timed(runner, calls_for_step, n_steps, pre=None):
-        """calls_for_step(i) -> list of callables issued for step i (one per layer)."""
-        for i in range(W):
-            for c in calls_for_step(i):
+    R = rotation_groups(wl, a.l2)
+    use_graph = a.l2 == "rotate" and a.launch == "graph"
+    graph_info = {}
+
+    def timed(calls_for_step, n_steps, graph_ok=True):
+        """calls_for_step(j) -> callables issued for global step j (one per layer).
+        Returns the timed interval in ms (sum of the per-step intervals when flushing)."""
+        for j in range(W):
+            for c in calls_for_step(j):
                 c()
         barrier_sync()
+        if a.l2 == "flush":
+            t0 = time.time()
+            evs = []
+            for i in range(n_steps):
+                flush_l2()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for c in calls_for_step(W + i):
+                    c()
+                e1.record()
+                evs.append((e0, e1))
+            barrier_sync()
+            sampler.mark(t0, time.time())
+            return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+        g = None
+        if use_graph and graph_ok:
+            g = torch.cuda.CUDAGraph()
+            cs = torch.cuda.Stream()
+            cs.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(cs):
+                g.capture_begin(capture_error_mode="thread_local")
+                for i in range(n_steps):
+                    for c in calls_for_step(W + i):
+                        c()
+                g.capture_end()
+            torch.cuda.current_stream().wait_stream(cs)
+            graph_info["uploaded"] = graph_upload(g, torch.cuda.current_stream())
+            barrier_sync()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
         t0 = time.time()
-        evs = []
-        for i in range(n_steps):
-            flush_l2()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for c in calls_for_step(W + i):
-                c()
-            e1.record()
-            evs.append((e0, e1))
+        e0.record()
+        if g is not None:
+            g.replay()
+        else:
+            for i in range(n_steps):
+                for c in calls_for_step(W + i):
+                    c()
+        e1.record()
         barrier_sync()
         sampler.mark(t0, time.time())
-        ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+        ms = e0.elapsed_time(e1)
+        del g
         return ms
 
     # ---- deferred (the product path) ----
-    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v)
+    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v, n_groups=R)
     r.load_initial_state()
     r.run_presteps()
     dev_inputs = [[r.device_inputs(x) for x in per_layer] for per_layer in host_inputs]
     outs = [torch.empty(wl.batch, wl.n_heads, wl.d_v, dtype=torch.float32, device=dev)
             for _ in range(wl.n_layers)]
-    prepared = [[dl.PreparedStep("decode", r.pool, l, r.slots, x["q"], x["k"], x["v"], x["lam"],
-                                 x["beta"], outs[l], wl.lambda_const) for l, x in enumerate(per_layer)]
-                for per_layer in dev_inputs]
 
     def check(st):
         if st != 0:
             raise dl.DeltaLogError(st, "dl_decode_step")
 
-    calls = lambda i: [(lambda p=p: check(p())) for p in prepared[i % ndist]]
-    ms = timed(r, calls, K)
+    def prepared_calls(kind, runner, cache):
+        """Step j: group j mod R, step inputs j mod ndist (argument blocks built once)."""
+        def calls(j):
+            key = (j % R, j % ndist)
+            if key not in cache:
+                g, t = key
+                cache[key] = [dl.PreparedStep(kind, runner.pool, l, runner.group_slots[g], x["q"], x["k"],
+                                              x["v"], x["lam"], x["beta"], outs[l], wl.lambda_const)
+                              for l, x in enumerate(dev_inputs[t])]
+            return [(lambda p=p: check(p())) for p in cache[key]]
+        return calls
+
+    total_ms = timed(prepared_calls("decode", r, {}), K)
     assert r.errors() == 0, "device error bits set during the benchmark"
-    total_ms = sum(ms)
     max_ms = reduce_max(total_ms)
     value = whole_job_rate(wl.units_per_step * K, world, max_ms)
 
-    # algorithmic bytes of the timed launches: slot b enters timed step i with
-    # c = (offset_b + W + i) mod L live entries (auto-merge cycle of length L)
+    # algorithmic bytes of the timed launches: each slot enters its step with the
+    # live entries of its own auto-merge cycle of length L
     offs = synth.slot_offsets(wl)
     bytes_total = 0.0
     for i in range(K):
-        c = (offs + W + i) % L
+        c = live_entries(offs, W + i, R, L)
         per_slot = [traffic.deferred_head_step(wl, int(cb), merge=(cb == L - 1)) for cb in c]
         bytes_total += sum(per_slot) * wl.n_heads * wl.n_layers
     launches = K * wl.n_layers
@@ -334,26 +436,25 @@ def run_gpu(a, wl, rank, world, dist):
             "avg_launch_us": round(total_ms * 1e3 / launches, 3),
             "frac_of_8tbs_spec": round(achieved_gbs / 8000.0, 4)}
 
-    result = {"value": value, "ms_per_step": max_ms / K, "roofline": roof, "gpu_launches": launches}
+    result = {"value": value, "ms_per_step": max_ms / K, "roofline": roof, "gpu_launches": launches,
+              "rotation_groups": R}
+    if use_graph:
+        result["graph_uploaded"] = graph_info.get("uploaded")
 
     # ---- eager comparison (same workload, full read-modify-write each step) ----
     if not a.no_eager:
-        re_ = DecodeRunner(wl, device=str(dev), mode="eager", tile_v=a.tile_v)
+        re_ = DecodeRunner(wl, device=str(dev), mode="eager", tile_v=a.tile_v, n_groups=R)
         re_.load_initial_state()
-        prep_e = [[dl.PreparedStep("eager", re_.pool, l, re_.slots, x["q"], x["k"], x["v"], x["lam"],
-                                   x["beta"], outs[l], wl.lambda_const) for l, x in enumerate(per_layer)]
-                  for per_layer in dev_inputs]
-        calls_e = lambda i: [(lambda p=p: check(p())) for p in prep_e[i % ndist]]
-        ms_e = timed(re_, calls_e, K)
+        ms_e = timed(prepared_calls("eager", re_, {}), K)
         assert re_.errors() == 0
-        tot_e = reduce_max(sum(ms_e))
+        tot_e = reduce_max(ms_e)
         eb = traffic.eager_head_step(wl) * wl.units_per_step * K
         result["eager"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_e),
                            "ms_per_step": tot_e / K,
                            "algorithmic_bytes_per_step": round(eb / K),
-                           "achieved_gbs": round(eb / (sum(ms_e) / 1e3) / 1e9, 1)}
+                           "achieved_gbs": round(eb / (ms_e / 1e3) / 1e9, 1)}
         result["deferred_bytes_per_step"] = round(bytes_total / K)
-        del re_, prep_e
+        del re_
         torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers ----
@@ -363,27 +464,29 @@ def run_gpu(a, wl, rank, world, dist):
         stage = [{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
                  for x in dev_inputs[0]]
         out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-        prep_2 = [dl.PreparedStep("decode", r.pool, l, r.slots, s["q"], s["k"], s["v"], s["lam"],
-                                  s["beta"], outs[l], wl.lambda_const) for l, s in enumerate(stage)]
+        prep_2 = [[dl.PreparedStep("decode", r.pool, l, gs, s["q"], s["k"], s["v"], s["lam"],
+                                   s["beta"], outs[l], wl.lambda_const) for l, s in enumerate(stage)]
+                  for gs in r.group_slots]
         h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
         d2h = sum(o.numel() * o.element_size() for o in outs)
 
-        def e2e_calls(i):
-            src = host_dev[i % ndist]
+        def e2e_calls(j):
+            src, prep = host_dev[j % ndist], prep_2[j % R]
             cs = []
             for l in range(wl.n_layers):
-                def one(l=l, src=src):
+                def one(l=l, src=src, prep=prep):
                     for k, v in src[l].items():
                         if v is not None:
                             stage[l][k].copy_(v, non_blocking=True)
-                    check(prep_2[l]())
+                    check(prep[l]())
                     out_host[l].copy_(outs[l], non_blocking=True)
                 cs.append(one)
             return cs
 
-        ms_2 = timed(r, e2e_calls, K)
+        # the call a user makes, launched directly (no graph)
+        ms_2 = timed(e2e_calls, K, graph_ok=False)
         assert r.errors() == 0
-        tot_2 = reduce_max(sum(ms_2))
+        tot_2 = reduce_max(ms_2)
         result["e2e"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_2), "unit": UNIT,
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "ms_per_step": tot_2 / K,
@@ -470,7 +573,7 @@ def run_reference(a, wl):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(wl, 1),
+            "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -517,10 +620,10 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; bf16 q/k/v, fp32 lambda/beta, fp32 state and log)",
-            "config": config_of(wl, world, a.tile_v), "roofline": res["roofline"],
+            "config": config_of(wl, world, a.tile_v, a.l2, a.launch), "roofline": res["roofline"],
             "gpu_launches": res["gpu_launches"],
             "hbm_tbs": res["roofline"]["achieved"] / 1e3}
-    for k in ("eager", "deferred_bytes_per_step", "e2e", "clocks"):
+    for k in ("eager", "deferred_bytes_per_step", "e2e", "clocks", "rotation_groups", "graph_uploaded"):
         if k in res:
             line[k] = res[k]
     if world == 1 and not a.no_cpu:

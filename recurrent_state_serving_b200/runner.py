@@ -9,6 +9,11 @@ subset of a larger pool when ``n_slots > batch``, to exercise non-contiguous ids
 Staggering (per-slot log fill offsets) is realised by untimed pre-steps: before
 the common steps, slot b takes ``offsets[b]`` decode steps with its own pre-step
 inputs, so slots reach their merge steps at different times.
+
+Slot groups: with ``n_groups = R > 1`` the pool holds R disjoint copies of the
+batch's slots (group g uses ids ``g * per_group + slots``), each prefilled and
+staggered the same way.  Stepping the groups in turn gives a working set R times
+one step's, for timing a batch whose own state fits in L2 without an L2 flush.
 """
 from __future__ import annotations
 
@@ -30,7 +35,7 @@ def _to_dev_input(a, in_dtype, device):
 class DecodeRunner:
     def __init__(self, wl: synth.Workload, *, n_slots: int | None = None, slot_seed: int | None = None,
                  layers=None, mode: str = "deferred", update: str | None = None,
-                 device: str = "cuda", tile_v: int = 0):
+                 device: str = "cuda", tile_v: int = 0, n_groups: int = 1):
         if mode not in ("deferred", "eager"):
             raise ValueError(mode)
         self.wl = wl
@@ -39,13 +44,17 @@ class DecodeRunner:
         self.device = torch.device(device)
         self.layers = list(range(wl.n_layers)) if layers is None else list(layers)
         n_slots = wl.batch if n_slots is None else n_slots
+        if n_groups < 1:
+            raise ValueError("n_groups must be >= 1")
         if slot_seed is None:
             ids = np.arange(wl.batch)
         else:
             ids = np.random.default_rng(slot_seed).permutation(n_slots)[:wl.batch]
         self.slot_ids = ids.astype(np.int32)
-        self.slots = torch.from_numpy(self.slot_ids).to(self.device)
-        self.pool = dl.Pool(n_slots, wl.n_layers, wl.n_heads, wl.d_k, wl.d_v, wl.log_cap,
+        self.group_slots = [torch.from_numpy((self.slot_ids + g * n_slots).astype(np.int32)).to(self.device)
+                            for g in range(n_groups)]
+        self.slots = self.group_slots[0]
+        self.pool = dl.Pool(n_slots * n_groups, wl.n_layers, wl.n_heads, wl.d_k, wl.d_v, wl.log_cap,
                             decay=wl.decay, update=self.update, n_kheads=wl.n_kheads,
                             device=device, with_log=(mode == "deferred"), tile_v=tile_v)
         self.offsets = synth.slot_offsets(wl)
@@ -55,8 +64,10 @@ class DecodeRunner:
         """Prefill: write each slot's initial state into the base, empty its log."""
         for layer in self.layers:
             S0 = torch.from_numpy(synth.initial_state(self.wl, layer)).to(self.device)
-            self.pool.state[self.slots.long(), layer] = S0
-        dl.dl_reset_slots(self.pool, self.slots)
+            for gs in self.group_slots:
+                self.pool.state[gs.long(), layer] = S0
+        for gs in self.group_slots:
+            dl.dl_reset_slots(self.pool, gs)
 
     def device_inputs(self, inp: dict, rows=None) -> dict:
         if rows is not None:
@@ -81,10 +92,11 @@ class DecodeRunner:
         n = int(self.offsets.max()) if len(self.offsets) else 0
         for p in range(n):
             rows = np.nonzero(self.offsets > p)[0]
-            sl = self.slots[torch.from_numpy(rows).to(self.device)]
+            sel = torch.from_numpy(rows).to(self.device)
             for layer in self.layers:
                 x = self.device_inputs(synth.step_inputs(self.wl, p, layer, prestep=True), rows)
-                self.call(layer, x, slots=sl)
+                for gs in self.group_slots:
+                    self.call(layer, x, slots=gs[sel])
 
     def materialize(self, layer: int) -> torch.Tensor:
         if self.mode == "eager":

@@ -49,3 +49,31 @@ def test_cycle_byte_accounting_matches_the_model():
     # the merge step moves the state twice, an append step once
     assert traffic.deferred_head_step(wl, L - 1, True) - traffic.deferred_head_step(wl, L - 1, False) == \
         pytest.approx(4 * wl.d_k * wl.d_v - traffic.entry_bytes(wl))
+
+
+def test_rotation_groups_cover_three_l2_sizes():
+    """Rotation: the groups' base states total >= 384 MiB, and one group fewer would not."""
+    for wl in (synth.GLA_DIAG, synth.GDN_GVA, synth.RETNET.with_(batch=1), synth.RETNET.with_(batch=16),
+               synth.KDA):
+        R = bench.rotation_groups(wl, "rotate")
+        step = wl.units_per_step * traffic.state_bytes(wl)
+        assert R * step >= bench.ROTATE_MIN_BYTES
+        assert R == 1 or (R - 1) * step < bench.ROTATE_MIN_BYTES
+        assert bench.rotation_groups(wl, "flush") == 1
+    assert bench.rotation_groups(synth.GLA_DIAG, "rotate") == 6      # 64 MiB per step
+    assert bench.rotation_groups(synth.GDN_GVA, "rotate") == 192     # 2 MiB per step
+    assert bench.rotation_groups(synth.KDA, "rotate") == 1
+
+
+def test_live_entries_follow_each_group_cycle():
+    """Group g is stepped at j = g, g + R, ...; before step j it has taken j // R steps."""
+    import numpy as np
+    offs = np.array([0, 3, 7])
+    L, R = 8, 3
+    seen = {g: 0 for g in range(R)}
+    for j in range(40):
+        g = j % R
+        np.testing.assert_array_equal(bench.live_entries(offs, j, R, L), (offs + seen[g]) % L)
+        seen[g] += 1
+    # one group: the plain per-step cycle
+    np.testing.assert_array_equal(bench.live_entries(offs, 13, 1, L), (offs + 13) % L)
