@@ -5,27 +5,39 @@
 // forms the head's key-side replay coefficients (DeltaLog paper, Section 3.3,
 // computed once per slot-head pair), streams the head's 64 KB base state, writes
 // o_t and the log entry, and -- as the only owner -- commits the shared log
-// metadata.  No CTA-wide barrier exists: the eight warps of a CTA work on eight
-// independent heads, so one head's latencies hide behind the others.
+// metadata.  No CTA-wide barrier exists inside the work loop: the eight warps of
+// a CTA work on independent heads, so one head's latencies hide behind the others.
 //
 // Lane l owns rows 4l..4l+3 for the key-side vectors (q, k, lbar_t, a_i,
-// Lambda_i) and columns 4l..4l+3 for the value side (v, b_i, o_t, and the
+// Lambda_i, A'_i) and columns 4l..4l+3 for the value side (v, b_i, o_t, and the
 // mat-vec accumulators).  The mat-vecs S^T qt and S^T kt need every row's qt/kt
 // in every lane: they come from the owning lane by warp shuffle, so each lane
 // accumulates its four columns over all 128 rows with no cross-lane reduction.
-// Replay dot products (q^T a_i, k^T a_i) are warp butterfly sums.
+// Replay dot products (q^T A'_i, k^T A'_i) are warp butterfly sums.
 //
-// Base-state streaming: each warp has its own ring of NSW shared-memory stages of
-// 8 KB (16 contiguous rows).  Lane 0 keeps NSW chunks in flight with
-// cp.async.bulk (TMA bulk copies, mbarrier complete_tx), running ahead from one
-// head into the warp's next head, whose slot id is read one head early.  A merge
-// step streams the tile twice: pass 1 for the mat-vecs, pass 2 -- an L2 hit,
-// the pass-1 copies ask L2 to keep the lines -- to write back the materialised
-// state S_t = e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T.
+// One stream per warp.  Each warp has a ring of NSW shared-memory stages of 8 KB;
+// lane 0 keeps NSW copies in flight with cp.async.bulk (TMA bulk copies, mbarrier
+// complete_tx), running ahead from one head into the warp's next head.  A head's
+// stream is
+//     its live log entries, newest first, EPC whole entries per stage,
+//     its base state, 16 rows per stage (pass 1: the mat-vecs),
+//     its base state again (pass 2), on a merge step under the delta rule,
+// so the replay reads entries from shared memory instead of waiting on one load
+// after another, and the newest entry -- whose Lambda is lbar -- arrives first.
+//
+// Merge step (the slot's L-th step): S_t = e^{lbar_t} (.) Sbar + sum_{i<c} A'_i b_i^T
+// + k_t b_t^T with A'_i = a_i (.) e^{lbar_t - Lambda_i}.  While replaying, the warp
+// also stores A'_i (its rows) and b_i (its columns) of up to TM_ENT entries into its
+// share of tensor memory (TMEM, 256 columns x 32 lanes per warp).  Without the delta
+// rule b_t = v_t is known from the start, so the new rows are written during pass 1
+// itself: the tile is read once and written once.  Under the delta rule b_t needs
+// all of pass 1, so the rows are written in pass 2, which re-reads the tile from L2
+// (pass-1 copies ask L2 to keep it).  Logs longer than TM_ENT entries (log_cap > 32)
+// merge in rounds of MRB entries staged in shared memory instead.
 //
 // Every wait is bounded (100 ms); a warp whose wait runs out sets
 // DL_EBIT_TIMEOUT, stops, and waits (bounded again) for its own copies still in
-// flight before it exits.
+// flight before the CTA frees its tensor memory and exits.
 #pragma once
 
 #include "dl_kernels.cuh"
@@ -42,13 +54,29 @@ constexpr uint32_t CB = CF * 4;             // 8 KB
 constexpr int NW = 8;                       // warps (heads in flight) per CTA
 constexpr int NTHREADS = NW * 32;
 constexpr int NSW = 3;                      // stages per warp
-constexpr int RPB = 4;                      // log entries per ReplayPrep load block
+constexpr int RPB = 4;                      // log entries per load block (merge rounds)
 constexpr int MRB = CF / (DK + DV);         // entries per merge round (A' and b in one stage)
 constexpr uint64_t WAIT_NS = 100000000ull;  // bound on every wait
 constexpr int NB = NSW + 2;                 // mbarriers per warp: stream stages + merge re-stream
+constexpr int TM_ENT = 32;                  // merge entries staged in TMEM per warp
+constexpr uint32_t TM_COLS = 512;           // TMEM columns per CTA (all of them)
+constexpr uint32_t TM_WCOLS = 256;          // per warp: two warps share each lane quarter
 constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * NB * 8 + 16;
-static_assert(NSW == 3, "the merge write-back uses stages 0-1 for the tile and stage 2 as scratch");
+static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
+static_assert(TM_ENT * 8 <= (int)TM_WCOLS, "A'_i and b_i take 8 columns per entry");
 constexpr unsigned FULL = 0xffffffffu;
+
+// A log entry as copied into shared memory: [a | b | Lambda] for per-key decay
+// (the whole ring row), [a | b | Lambda_0 and 3 pad floats] for scalar decay,
+// [a | b] without decay.  EPC entries fill one stage.
+template <int DECAY>
+struct LogCopy {
+    static constexpr uint32_t ESB = DECAY == DL_DECAY_DIAG     ? (2 * DK + DV) * 4
+                                    : DECAY == DL_DECAY_SCALAR ? (DK + DV + 4) * 4
+                                                               : (DK + DV) * 4;
+    static constexpr int ESF = ESB / 4;
+    static constexpr int EPC = CB / ESB;
+};
 
 template <typename T> __device__ __forceinline__ void load4(const T *p, float (&v)[4]);
 template <> __device__ __forceinline__ void load4<float>(const float *p, float (&v)[4]) {
@@ -69,32 +97,58 @@ __device__ __forceinline__ float warp_allsum(float x) {
     return x;
 }
 
+enum MergeKind : int {
+    MK_APPEND = 0,  // append step: o_t from base + log, entry c appended
+    MK_FUSED = 1,   // merge without the delta rule: new rows written during pass 1
+    MK_PASS2 = 2,   // merge under the delta rule: new rows written in pass 2
+    MK_ROUNDS = 3   // merge of more than TM_ENT entries: rounds staged in shared memory
+};
+
 // One head as the warp sees it.
 struct Head {
     int it;        // work item (batch row * H + head), n_items when past the end
     int s;         // slot id
+    int ok;        // slot id in range (the head is processed unless st is set later)
     int c;         // live entries
     int st;        // 0, or the error bit that makes the head skipped
-    int n;         // chunks in its stream: 0 (bad slot), 8, or 16 (merge / eager)
-    int merge;     // merge step (or eager step)
+    int mk;        // MergeKind
+    int nl;        // log chunks in its stream
+    int n;         // stream positions: nl + NCH (+ NCH for MK_PASS2); 0 when skipped
     size_t head;   // (slot, layer, head) index
 };
 
 template <int DECAY, bool DELTA, typename IT>
 __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 {
+    using LC = LogCopy<DECAY>;
+    constexpr uint32_t ESB = LC::ESB;
+    constexpr int ESF = LC::ESF, EPC = LC::EPC;
+
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     float *st = reinterpret_cast<float *>(smem) + (size_t)w * NSW * CF;
     uint64_t *fb = reinterpret_cast<uint64_t *>(smem + (size_t)NW * NSW * CB) + w * NB;
-    uint64_t *pb = fb + NSW;  // merge write-back: tile re-stream through stages 0 and 1
+    uint64_t *pb = fb + NSW;  // round-wise merge: tile re-stream through stages 0 and 1
     int *next_k = reinterpret_cast<int *>(smem + (size_t)NW * NSW * CB + (size_t)NW * NB * 8);
+    uint32_t *tm_slot = reinterpret_cast<uint32_t *>(next_k + 1);
+
+    // merges with live entries need tensor memory (auto-merge decode steps only)
+    const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
     if (lane == 0) {
         for (int s = 0; s < NB; ++s) ptx::mbar_init(&fb[s], 1);
         ptx::fence_barrier_init();
     }
     if (threadIdx.x == 0) *next_k = NW;  // warp w starts with the CTA's w-th head
+    if (use_tm && w == 0) {
+        ptx::tmem_alloc(tm_slot, TM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tmem_fence_before_sync();
     __syncthreads();
+    ptx::tmem_fence_after_sync();
+    // this warp's TMEM: lanes of its quarter, columns of its half
+    const uint32_t tm = use_tm ? *tm_slot + ((uint32_t)(32 * (w & 3)) << 16) + TM_WCOLS * (uint32_t)(w >> 2)
+                               : 0u;
 
     const int n_items = p.batch * p.H;
     const int G = gridDim.x;
@@ -111,93 +165,110 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     const uint64_t pol_stream = ptx::policy_evict_first();
     const uint64_t pol_keep = ptx::policy_evict_last();
 
-    // -- head metadata: slot id first (it locates the tile and lets the first
-    //    chunks go out), live length after (it decides append or merge)
+    // -- head metadata: slot id first (it locates the tile and the log), live
+    //    length after (it sizes the log part of the stream and decides the merge)
     auto slot_of = [&](int it) -> int { return it < n_items ? p.slots[it / p.H] : -1; };
     auto len_of = [&](const Head &hd) -> int {
-        return (hd.n && p.log_len) ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
+        return (hd.ok && p.log_len) ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
     };
     auto resolve_slot = [&](Head &hd, int it, int s) {
         hd.it = it;
         hd.s = s;
+        hd.ok = 0;
         hd.c = 0;
         hd.st = 0;
-        hd.merge = 0;
-        hd.head = 0;
+        hd.mk = MK_APPEND;
+        hd.nl = 0;
         hd.n = 0;
+        hd.head = 0;
         if (it >= n_items) return;
         if (s < 0 || s >= p.n_slots) { hd.st = DL_EBIT_SLOT_RANGE; return; }
         hd.head = ((size_t)s * p.n_layers + p.layer) * p.H + (it % p.H);
-        hd.n = NCH;  // pass 1 never depends on the live length
+        hd.ok = 1;
     };
     auto resolve_len = [&](Head &hd, int c) {
-        if (!hd.n) return;
+        if (!hd.ok) return;
         hd.c = c;
         if (p.eager) {
-            if (hd.c != 0) hd.st = DL_EBIT_LIVE_LOG;
-        } else if (hd.c < 0 || hd.c > p.L) {
+            if (c != 0) hd.st = DL_EBIT_LIVE_LOG;
+        } else if (c < 0 || c > p.L) {
             hd.st = DL_EBIT_LOG_LEN;
-        } else if (!(p.auto_merge && hd.c >= p.L - 1) && hd.c >= p.L) {
+        } else if (!(p.auto_merge && c >= p.L - 1) && c >= p.L) {
             hd.st = DL_EBIT_LOG_FULL;
         }
-        hd.merge = p.eager || (p.auto_merge && hd.c >= p.L - 1);
-        hd.n = NCH;
+        if (hd.st) return;
+        const bool merge = p.eager || (p.auto_merge && c >= p.L - 1);
+        hd.mk = !merge ? MK_APPEND : c > TM_ENT ? MK_ROUNDS : DELTA ? MK_PASS2 : MK_FUSED;
+        hd.nl = (c + EPC - 1) / EPC;
+        hd.n = hd.nl + NCH + (hd.mk == MK_PASS2 ? NCH : 0);
     };
-    // L2 warm-up of what the warp reads for a head besides its base state
-    auto warm = [&](const Head &hd) {
-        if (lane != 0 || hd.it >= n_items || hd.st) return;
-        const int bi = hd.it / p.H, h = hd.it % p.H, gk = h / (p.H / p.Hk);
+    // L2 warm-up of a head's token rows (they depend on the work item only)
+    auto warm_token = [&](int it) {
+        if (lane != 0 || it >= n_items) return;
+        const int bi = it / p.H, h = it % p.H, gk = h / (p.H / p.Hk);
         ptx::prefetch_l2(static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + gk) * DK, DK * sizeof(IT));
         ptx::prefetch_l2(static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + gk) * DK, DK * sizeof(IT));
         ptx::prefetch_l2(static_cast<const IT *>(p.v) + ((size_t)bi * p.H + h) * DV, DV * sizeof(IT));
         if (DECAY == DL_DECAY_DIAG && !p.lam_const)
             ptx::prefetch_l2(p.lam + ((size_t)bi * p.H + h) * DK, DK * 4);
-        if (hd.c > 0) ptx::prefetch_l2(p.log + hd.head * (size_t)p.L * E, (uint32_t)(hd.c * E * 4));
     };
 
-    // -- the warp's chunk stream: positions [base, base + cur.n) belong to cur,
-    //    then up to NCH pass-1 chunks of nxt (its live length may not be known yet)
+    // -- the warp's stream: positions [base, base + cur.n) belong to cur, then up to
+    //    nxt.n positions of nxt (issued once nxt's live length is known)
     int gc = 0, gi = 0, base = 0;  // consumed / issued stream positions
     bool abort = false;
-    uint32_t pph = 0u;             // merge re-stream barrier phases (bit b: barrier pb[b])
-    uint32_t pb_pend = 0u;         // merge re-stream copies in flight (bit b)
+    uint32_t pph = 0u;             // round-wise merge re-stream barrier phases (bit b: pb[b])
+    uint32_t pb_pend = 0u;         // round-wise merge re-stream copies in flight (bit b)
     Head cur, nxt;
+    nxt.ok = 0;
+    nxt.n = 0;
     const int it0 = (long long)blockIdx.x + (long long)w * G < n_items ? blockIdx.x + w * G : n_items;
+    warm_token(it0);
     resolve_slot(cur, it0, slot_of(it0));
     int it_nxt = grab();                 // the warp's next head, and its slot id, one head early
     int s_nxt = slot_of(it_nxt);
-    bool nxt_res = false;                // nxt's live length (hence merge or not) known
+    bool nxt_res = false;                // nxt's live length known
+    int c_nxt = 0;
 
+    // position x of head hd into stage gi % NSW (lane 0)
+    auto issue_pos = [&](const Head &hd, int x) {
+        const int sg = gi % NSW;
+        uint64_t *bar = &fb[sg];
+        float *dst = st + (size_t)sg * CF;
+        if (x < hd.nl) {
+            const int hi = hd.c - EPC * x, lo = hi - EPC > 0 ? hi - EPC : 0;
+            const float *src = p.log + hd.head * (size_t)p.L * E;
+            ptx::mbar_arrive_expect_tx(bar, (uint32_t)(hi - lo) * ESB);
+            if (DECAY == DL_DECAY_DIAG) {
+                ptx::bulk_g2s(dst, src + (size_t)lo * E, (uint32_t)(hi - lo) * ESB, bar, pol_stream);
+            } else {
+                for (int i = lo; i < hi; ++i)
+                    ptx::bulk_g2s(dst + (size_t)(i - lo) * ESF, src + (size_t)i * E, ESB, bar, pol_stream);
+            }
+        } else {
+            const int y = x - hd.nl;
+            const bool keep = y < NCH && (hd.mk == MK_PASS2 || hd.mk == MK_ROUNDS);
+            ptx::mbar_arrive_expect_tx(bar, CB);
+            ptx::bulk_g2s(dst, p.state + hd.head * (size_t)(DK * DV) + (size_t)(y & (NCH - 1)) * CF, CB, bar,
+                          keep ? pol_keep : pol_stream);
+        }
+    };
     auto issue_upto = [&](int limit) {
         while (gi < limit) {
-            const Head *hd;
-            int x;
             if (gi < base + cur.n) {
-                hd = &cur;
-                x = gi - base;
-            } else {
-                // a merge head needs its stages as scratch after pass 1: no look-ahead
-                const int rel = gi - base - cur.n;
-                const int nit = it_nxt;
-                const bool ok = !(cur.merge && cur.st == 0) && nit < n_items && s_nxt >= 0 &&
-                                s_nxt < p.n_slots && rel < NCH;
-                if (!ok) break;
-                if (lane == 0) {
-                    const size_t hn = ((size_t)s_nxt * p.n_layers + p.layer) * p.H + (nit % p.H);
-                    const int sg = gi % NSW;
-                    ptx::mbar_arrive_expect_tx(&fb[sg], CB);
-                    ptx::bulk_g2s(st + (size_t)sg * CF, p.state + hn * (size_t)(DK * DV) + (size_t)rel * CF,
-                                  CB, &fb[sg], (nxt_res && nxt.merge) ? pol_keep : pol_stream);
-                }
+                if (lane == 0) issue_pos(cur, gi - base);
                 ++gi;
                 continue;
             }
-            if (lane == 0) {
-                const int sg = gi % NSW;
-                ptx::mbar_arrive_expect_tx(&fb[sg], CB);
-                ptx::bulk_g2s(st + (size_t)sg * CF, p.state + hd->head * (size_t)(DK * DV) + (size_t)x * CF,
-                              CB, &fb[sg], hd->merge ? pol_keep : pol_stream);
+            // a round-wise merge needs its stages as scratch after pass 1: no look-ahead
+            if ((cur.mk == MK_ROUNDS && cur.st == 0) || !nxt.ok) break;
+            if (!nxt_res) {
+                resolve_len(nxt, c_nxt);
+                nxt_res = true;
             }
+            const int rel = gi - base - cur.n;
+            if (rel >= nxt.n) break;
+            if (lane == 0) issue_pos(nxt, rel);
             ++gi;
         }
     };
@@ -214,9 +285,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         issue_upto(gc + NSW);
     };
 
-    issue_upto(NSW);
+    // The first head has no head before it to hide its prologue.  Its dependent
+    // loads (slot id, then live length) go out before any of its stream does.
     resolve_len(cur, len_of(cur));
-    warm(cur);
+    issue_upto(NSW);
+
     // Finalize of the previous head, checked one head later so the atomic's round
     // trip overlaps the next head's work
     int fin_old = -1, fin_len = 0;
@@ -231,21 +304,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
     while (cur.it < n_items) {
         // the next head: slot id read one head ago; its live length is loaded now
-        // and looked at after this head's pass 1
+        // and used when the stream reaches it
         resolve_slot(nxt, it_nxt, s_nxt);
         nxt_res = false;
-        const int c_nxt = len_of(nxt);
+        c_nxt = len_of(nxt);
+        if (nxt.ok) warm_token(nxt.it);
         if (cur.st && lane == 0) atomicOr(p.err, cur.st);
 
         if (cur.st == 0) {
-            const int c = cur.c;
-            const bool merge_now = cur.merge != 0;
+            const int c = cur.c, mk = cur.mk;
             const int bi = cur.it / p.H, h = cur.it % p.H;
             const size_t row = (size_t)bi * p.H + h;
             const size_t sl = (size_t)cur.s * p.n_layers + p.layer;
             float *tile = p.state + cur.head * (size_t)(DK * DV);
             float *ring = p.log ? p.log + cur.head * (size_t)p.L * E : nullptr;
             const int gk = h / (p.H / p.Hk);
+            const bool stage_tm = use_tm && c > 0 && (mk == MK_FUSED || mk == MK_PASS2);
 
             // -- token, cumulative log-decay and prescale (rows 4l..4l+3)
             float q_own[4], k_own[4], v_own[4], lam[4] = {0.f, 0.f, 0.f, 0.f};
@@ -258,15 +332,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (DECAY == DL_DECAY_DIAG) {
                 const float4 l4 = ldg4(p.lam + (p.lam_const ? (size_t)h : row) * DK + 4 * lane);
                 lam[0] = l4.x; lam[1] = l4.y; lam[2] = l4.z; lam[3] = l4.w;
-                if (c > 0) {
-                    const float4 p4 = ldg4(ring + (size_t)(c - 1) * E + DK + DV + 4 * lane);
-                    lp[0] = p4.x; lp[1] = p4.y; lp[2] = p4.z; lp[3] = p4.w;
-                }
             } else if (DECAY == DL_DECAY_SCALAR) {
                 const float ls = __ldg(p.lam + (p.lam_const ? (size_t)h : row));
-                const float ps = c > 0 ? __ldg(ring + (size_t)(c - 1) * E + DK + DV) : 0.f;
 #pragma unroll
-                for (int x = 0; x < 4; ++x) { lam[x] = ls; lp[x] = ps; }
+                for (int x = 0; x < 4; ++x) lam[x] = ls;
+            }
+            // lbar = Lambda of the newest entry, the last row of the first log chunk
+            if (c > 0) {
+                if (!wait_chunk()) { abort = true; break; }
+                const int lo0 = c - EPC > 0 ? c - EPC : 0;
+                const float *ent = st + (size_t)(gc % NSW) * CF + (size_t)(c - 1 - lo0) * ESF + DK + DV;
+                if (DECAY == DL_DECAY_DIAG) {
+                    const float4 p4 = reinterpret_cast<const float4 *>(ent)[lane];
+                    lp[0] = p4.x; lp[1] = p4.y; lp[2] = p4.z; lp[3] = p4.w;
+                } else if (DECAY == DL_DECAY_SCALAR) {
+                    const float ps = ent[0];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) lp[x] = ps;
+                }
             }
             float ell[4], e_own[4], qt[4], kt[4];
             float kq = 0.f;
@@ -281,58 +364,101 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
             kq = warp_allsum(kq);
 
-            // -- ReplayPrep + value replay: Y += (q^T A'_i) b_i, (k^T A'_i) b_i, eight
-            //    entries' loads in flight at a time
+            // -- ReplayPrep + value replay over the log chunks (newest first):
+            //    Y += (q^T A'_i) b_i, (k^T A'_i) b_i; a merge also stages A'_i, b_i in TMEM
             float4 Yq = make_float4(0.f, 0.f, 0.f, 0.f), Yk = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int i0 = 0; i0 < c; i0 += RPB) {
-                float4 A[RPB], B[RPB], Lq[RPB];
+            for (int x = 0; x < cur.nl; ++x) {
+                if (x > 0 && !wait_chunk()) { abort = true; break; }
+                const float *sb = st + (size_t)(gc % NSW) * CF;
+                const int hi = c - EPC * x, lo = hi - EPC > 0 ? hi - EPC : 0;
+                float pq[EPC], pk[EPC];
 #pragma unroll
-                for (int u = 0; u < RPB; ++u) {
-                    if (i0 + u < c) {
-                        const float *ent = ring + (size_t)(i0 + u) * E;
-                        A[u] = ldg4(ent + 4 * lane);
-                        B[u] = ldg4(ent + DK + 4 * lane);
+                for (int e = 0; e < EPC; ++e) {
+                    pq[e] = 0.f;
+                    pk[e] = 0.f;
+                    if (lo + e < hi) {
+                        const float *ent = sb + (size_t)e * ESF;
+                        const float4 a4 = reinterpret_cast<const float4 *>(ent)[lane];
+                        float Lv[4] = {0.f, 0.f, 0.f, 0.f};
                         if (DECAY == DL_DECAY_DIAG) {
-                            Lq[u] = ldg4(ent + DK + DV + 4 * lane);
-                        } else {
-                            const float Ls = DECAY == DL_DECAY_SCALAR ? __ldg(ent + DK + DV) : 0.f;
-                            Lq[u] = make_float4(Ls, Ls, Ls, Ls);
+                            const float4 L4 = reinterpret_cast<const float4 *>(ent + DK + DV)[lane];
+                            Lv[0] = L4.x; Lv[1] = L4.y; Lv[2] = L4.z; Lv[3] = L4.w;
+                        } else if (DECAY == DL_DECAY_SCALAR) {
+                            const float Ls = ent[DK + DV];
+#pragma unroll
+                            for (int y = 0; y < 4; ++y) Lv[y] = Ls;
                         }
-                    }
-                }
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+                        float wq[4];
 #pragma unroll
-                for (int u = 0; u < RPB; ++u) {
-                    if (i0 + u < c) {
-                        const float av[4] = {A[u].x, A[u].y, A[u].z, A[u].w};
-                        const float Lv[4] = {Lq[u].x, Lq[u].y, Lq[u].z, Lq[u].w};
-                        float pq = 0.f, pk = 0.f;
-#pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            const float g = DECAY == DL_DECAY_NONE ? 1.f : expf(ell[x] - Lv[x]);
-                            const float wq = av[x] * g;
-                            pq = fmaf(wq, q_own[x], pq);
+                        for (int y = 0; y < 4; ++y) {
+                            const float g = DECAY == DL_DECAY_NONE ? 1.f : expf(ell[y] - Lv[y]);
+                            wq[y] = av[y] * g;
+                            pq[e] = fmaf(wq[y], q_own[y], pq[e]);
                             if (DELTA) {
                                 const float wk = (p.undecayed && DECAY != DL_DECAY_NONE)
-                                                     ? av[x] * expf(lp[x] - Lv[x]) : wq;
-                                pk = fmaf(wk, k_own[x], pk);
+                                                     ? av[y] * expf(lp[y] - Lv[y]) : wq[y];
+                                pk[e] = fmaf(wk, k_own[y], pk[e]);
                             }
                         }
-                        pq = warp_allsum(pq);
-                        fma4(Yq, pq, B[u]);
-                        if (DELTA) {
-                            pk = warp_allsum(pk);
-                            fma4(Yk, pk, B[u]);
+                        if (stage_tm) {
+                            const float4 b4 = reinterpret_cast<const float4 *>(ent + DK)[lane];
+                            const float tv[8] = {wq[0], wq[1], wq[2], wq[3], b4.x, b4.y, b4.z, b4.w};
+                            ptx::tmem_st8(tm + 8u * (uint32_t)(lo + e), tv);
                         }
                     }
                 }
+                // butterfly sums of the chunk's entries, level by level
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) {
+                        pq[e] += __shfl_xor_sync(FULL, pq[e], o);
+                        if (DELTA) pk[e] += __shfl_xor_sync(FULL, pk[e], o);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) {
+                    if (lo + e < hi) {
+                        const float4 b4 = reinterpret_cast<const float4 *>(sb + (size_t)e * ESF + DK)[lane];
+                        fma4(Yq, pq[e], b4);
+                        if (DELTA) fma4(Yk, pk[e], b4);
+                    }
+                }
+                release();
             }
+            if (abort) break;
+            if (stage_tm) ptx::tmem_wait_st();
 
-            // the next head's phase is known from here on (its chunks' L2 policy)
-            resolve_len(nxt, c_nxt);
-            nxt_res = true;
-            warm(nxt);
+            // new rows of one 16-row block of the merged state from its Sbar rows in
+            // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending
+            auto write_rows = [&](const float *sb, int cx, const float4 &bt4) {
+                float4 acc[CR];
+#pragma unroll
+                for (int rr = 0; rr < CR; ++rr) {
+                    const float4 S = reinterpret_cast<const float4 *>(sb + rr * DV)[lane];
+                    const float e = __shfl_sync(FULL, e_own[rr & 3], 4 * cx + (rr >> 2));
+                    acc[rr] = make_float4(S.x * e, S.y * e, S.z * e, S.w * e);
+                }
+                const int nj = stage_tm ? c : 0;  // TMEM is read only where it was written
+                for (int j = 0; j < nj; ++j) {
+                    float tv[8];
+                    ptx::tmem_ld8(tm + 8u * (uint32_t)j, tv);
+                    const float4 b4 = make_float4(tv[4], tv[5], tv[6], tv[7]);
+#pragma unroll
+                    for (int rr = 0; rr < CR; ++rr)
+                        fma4(acc[rr], __shfl_sync(FULL, tv[rr & 3], 4 * cx + (rr >> 2)), b4);
+                }
+#pragma unroll
+                for (int rr = 0; rr < CR; ++rr) {
+                    fma4(acc[rr], __shfl_sync(FULL, k_own[rr & 3], 4 * cx + (rr >> 2)), bt4);
+                    __stcs(reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane, acc[rr]);
+                }
+            };
 
-            // -- AppendDecode pass 1: y_q = Sbar^T qt, y_k = Sbar^T kt (columns 4l..4l+3)
+            // -- AppendDecode pass 1: y_q = Sbar^T qt, y_k = Sbar^T kt (columns 4l..4l+3);
+            //    without the delta rule a merge writes its new rows here as well
+            const float4 v4 = make_float4(v_own[0], v_own[1], v_own[2], v_own[3]);
             for (int cx = 0; cx < NCH; ++cx) {
                 if (!wait_chunk()) { abort = true; break; }
                 const float *sb = st + (size_t)(gc % NSW) * CF;
@@ -343,13 +469,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     fma4(Yq, __shfl_sync(FULL, qt[rr & 3], src), S);
                     if (DELTA) fma4(Yk, __shfl_sync(FULL, kt[rr & 3], src), S);
                 }
+                if (!DELTA && mk == MK_FUSED) write_rows(sb, cx, v4);
                 release();
             }
             if (abort) break;
 
             finish_commit();
 
-            // -- b_t, o_t, and the append (entry c) or the merge-step write-back
+            // -- b_t, o_t, and the append (entry c)
             const float yq[4] = {Yq.x, Yq.y, Yq.z, Yq.w}, yk[4] = {Yk.x, Yk.y, Yk.z, Yk.w};
             float bt[4], o[4];
 #pragma unroll
@@ -360,17 +487,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             const float4 bt4 = make_float4(bt[0], bt[1], bt[2], bt[3]);
             if (p.want_out)
                 *reinterpret_cast<float4 *>(p.out + row * DV + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-            if (!merge_now) {
+            if (mk == MK_APPEND) {
                 float *ent = ring + (size_t)c * E;
                 *reinterpret_cast<float4 *>(ent + DK + 4 * lane) = bt4;
                 *reinterpret_cast<float4 *>(ent + 4 * lane) = make_float4(k_own[0], k_own[1], k_own[2], k_own[3]);
                 if (DECAY == DL_DECAY_DIAG)
                     *reinterpret_cast<float4 *>(ent + DK + DV + 4 * lane) = make_float4(ell[0], ell[1], ell[2], ell[3]);
                 if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[DK + DV] = ell[0];
-            } else {
-                // Merge step: S_t = e^{lbar_t} (.) Sbar + sum_{i<=c} A'_i b_i^T, entry c being
-                // the token (A'_c = k, b_c = b_t).  Pass 1 left every stage idle (no
-                // look-ahead past a merge head).  Per round of up to MRB entries, stage 2
+            } else if (mk == MK_PASS2) {
+                // -- pass 2: the tile again (from L2), rewritten row block by row block
+                for (int cx = 0; cx < NCH; ++cx) {
+                    if (!wait_chunk()) { abort = true; break; }
+                    write_rows(st + (size_t)(gc % NSW) * CF, cx, bt4);
+                    release();
+                }
+                if (abort) break;
+            } else if (mk == MK_ROUNDS) {
+                // More entries than TMEM holds.  Pass 1 left every stage idle (no
+                // look-ahead past this head).  Per round of up to MRB entries, stage 2
                 // holds A' (this lane's rows) and b (its columns); the tile is re-streamed
                 // from L2 through stages 0/1 (Sbar in the first round, the previous round's
                 // partial sums after that) and rewritten row block by row block.
@@ -478,24 +612,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (!p.eager) {
                 if (lane == 0) fin_old = atomicAdd(p.arrive + sl, 1);
                 fin_sl = sl;
-                fin_len = merge_now ? 0 : c + 1;
+                fin_len = mk != MK_APPEND ? 0 : c + 1;
             }
         } else {
-            // skipped head: consume (and ignore) the chunks that were streamed for it
-            for (int x = 0; x < cur.n; ++x) {
-                if (!wait_chunk()) { abort = true; break; }
-                release();
-            }
-            if (abort) break;
-            resolve_len(nxt, c_nxt);
-            nxt_res = true;
-            warm(nxt);
+            // skipped head: nothing was streamed for it
             finish_commit();
         }
 
         // advance: nxt becomes cur; take the head after it and read its slot id
+        if (!nxt_res) resolve_len(nxt, c_nxt);
         base += cur.n;
         cur = nxt;
+        nxt.ok = 0;
+        nxt.n = 0;
         it_nxt = grab();
         s_nxt = slot_of(it_nxt);
         nxt_res = false;
@@ -509,7 +638,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         for (; gc < gi; ++gc) ptx::mbar_wait_bounded(&fb[gc % NSW], (gc / NSW) & 1, WAIT_NS);
         for (int b2 = 0; b2 < 2; ++b2)
             if ((pb_pend >> b2) & 1u) ptx::mbar_wait_bounded(&pb[b2], (pph >> b2) & 1u, WAIT_NS);
+        if (use_tm) ptx::tmem_wait_st();
     }
+    // tensor memory goes back once every warp is done with it
+    ptx::tmem_fence_before_sync();
+    __syncthreads();
+    ptx::tmem_fence_after_sync();
+    if (use_tm && w == 0) ptx::tmem_dealloc(*tm_slot, TM_COLS);
 }
 
 }  // namespace wh

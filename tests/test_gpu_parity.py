@@ -23,6 +23,19 @@ REDUCED = {
     "gdn_gva_256": synth.GDN_GVA.with_(batch=3, steps=256),
     "kda": synth.KDA.with_(n_layers=2, batch=3, n_heads=4, n_kheads=4, steps=256),
     "retnet": synth.RETNET.with_(n_layers=2, batch=7, n_heads=4, n_kheads=4, steps=256),
+    # 128 x 128 heads without decay (linear attention, DeltaNet)
+    "la_d128": synth.TINY_LA.with_(batch=3, n_heads=3, n_kheads=3, d_k=128, d_v=128, steps=96,
+                                   log_cap=12, qkv_std=1 / np.sqrt(128), init_std=0.02),
+    "deltanet_d128": synth.TINY_LA.with_(batch=3, n_heads=3, n_kheads=3, d_k=128, d_v=128, steps=96,
+                                         log_cap=12, qkv_std=1 / np.sqrt(128), init_std=0.02,
+                                         update="delta", k_l2norm=True),
+    # long logs: a merge of exactly 32 entries, and merges of more than 32 entries
+    "kda_L33": synth.KDA.with_(n_layers=1, batch=3, n_heads=3, n_kheads=3, steps=140, log_cap=33),
+    "gla_L64": synth.GLA_DIAG.with_(batch=2, n_heads=3, n_kheads=3, steps=200, log_cap=64,
+                                    staggered=True),
+    "retnet_L48": synth.RETNET.with_(n_layers=1, batch=3, n_heads=3, n_kheads=3, steps=160, log_cap=48),
+    "kda_L40": synth.KDA.with_(n_layers=1, batch=2, n_heads=3, n_kheads=3, steps=128, log_cap=40,
+                               staggered=True),
 }
 
 
@@ -44,7 +57,7 @@ def _tile_ok(wl, tile_v):
     if tile_v == 32:
         return wl.d_k >= 64 and wl.d_v % 32 == 0
     if tile_v == 128:
-        return wl.d_k == 128 and wl.d_v == 128 and wl.log_cap <= 32
+        return wl.d_k == 128 and wl.d_v == 128
     return True
 
 
