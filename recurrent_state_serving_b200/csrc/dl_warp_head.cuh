@@ -13,7 +13,9 @@
 // mat-vec accumulators).  The mat-vecs S^T qt and S^T kt need every row's qt/kt
 // in every lane: they come from the owning lane by warp shuffle, so each lane
 // accumulates its four columns over all 128 rows with no cross-lane reduction.
-// Replay dot products (q^T A'_i, k^T A'_i) are warp butterfly sums.
+// Replay dot products (q^T A'_i, k^T A'_i) are warp butterfly sums.  Values a
+// row block needs in every lane (qt, kt, e^{lbar_t}, k and A'_i of its 16 rows) are
+// read as shared-memory broadcasts from a small per-warp area the owning lanes fill.
 //
 // One stream per warp.  Each warp has a ring of NSW shared-memory stages of 8 KB;
 // lane 0 keeps NSW copies in flight with cp.async.bulk (TMA bulk copies, mbarrier
@@ -34,6 +36,13 @@
 // all of pass 1, so the rows are written in pass 2, which re-reads the tile from L2
 // (pass-1 copies ask L2 to keep it).  Logs longer than TM_ENT entries (log_cap > 32)
 // merge in rounds of MRB entries staged in shared memory instead.
+//
+// Order of work.  The CTA's heads are blockIdx.x + k * gridDim.x.  When there are more
+// of them than warps (and at most KMAX), the CTA first reads every head's slot id and
+// live length (all threads at once) and puts the merge steps first: a merge head
+// costs several append heads, and started early it overlaps their streaming instead
+// of ending the launch alone.  Warps then take heads in that order from a shared
+// counter.
 //
 // Every wait is bounded (100 ms); a warp whose wait runs out sets
 // DL_EBIT_TIMEOUT, stops, and waits (bounded again) for its own copies still in
@@ -61,7 +70,14 @@ constexpr int NB = NSW + 2;                 // mbarriers per warp: stream stages
 constexpr int TM_ENT = 32;                  // merge entries staged in TMEM per warp
 constexpr uint32_t TM_COLS = 512;           // TMEM columns per CTA (all of them)
 constexpr uint32_t TM_WCOLS = 256;          // per warp: two warps share each lane quarter
-constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * NB * 8 + 16;
+constexpr int AG = 4;                       // merge entries per TMEM load / shared-memory publish
+// per-warp scratch: the head's row vectors qt, kt, e^{lbar_t}, k, lbar_t (5 x 128 floats)
+// and the A' values of AG entries for the 16 rows of one block
+constexpr int WSCR = 5 * DK + AG * CR;
+// per-CTA head list: slot id, live length and the processing order of up to KMAX heads
+constexpr int KMAX = 512;
+constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4 + (size_t)NW * NB * 8 + 32 +
+                        (size_t)KMAX * (4 + 4 + 2);
 static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
 static_assert(TM_ENT * 8 <= (int)TM_WCOLS, "A'_i and b_i take 8 columns per entry");
 constexpr unsigned FULL = 0xffffffffu;
@@ -127,10 +143,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     float *st = reinterpret_cast<float *>(smem) + (size_t)w * NSW * CF;
-    uint64_t *fb = reinterpret_cast<uint64_t *>(smem + (size_t)NW * NSW * CB) + w * NB;
+    float *rv = reinterpret_cast<float *>(smem + (size_t)NW * NSW * CB) + (size_t)w * WSCR;
+    float *rv_qt = rv, *rv_kt = rv + DK, *rv_e = rv + 2 * DK, *rv_k = rv + 3 * DK, *rv_l = rv + 4 * DK;
+    float *ag = rv + 5 * DK;
+    unsigned char *bars = smem + (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4;
+    uint64_t *fb = reinterpret_cast<uint64_t *>(bars) + w * NB;
     uint64_t *pb = fb + NSW;  // round-wise merge: tile re-stream through stages 0 and 1
-    int *next_k = reinterpret_cast<int *>(smem + (size_t)NW * NSW * CB + (size_t)NW * NB * 8);
+    int *next_k = reinterpret_cast<int *>(bars + (size_t)NW * NB * 8);
     uint32_t *tm_slot = reinterpret_cast<uint32_t *>(next_k + 1);
+    int *cnt = next_k + 2;  // merge heads, next merge position, next other position
+    int *pre_slot = next_k + 8;
+    int *pre_len = pre_slot + KMAX;
+    uint16_t *order = reinterpret_cast<uint16_t *>(pre_len + KMAX);
 
     // merges with live entries need tensor memory (auto-merge decode steps only)
     const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
@@ -138,7 +162,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         for (int s = 0; s < NB; ++s) ptx::mbar_init(&fb[s], 1);
         ptx::fence_barrier_init();
     }
-    if (threadIdx.x == 0) *next_k = NW;  // warp w starts with the CTA's w-th head
+    if (threadIdx.x == 0) {
+        *next_k = NW;  // warp w starts with the CTA's w-th head
+        cnt[0] = cnt[1] = cnt[2] = 0;
+    }
     if (use_tm && w == 0) {
         ptx::tmem_alloc(tm_slot, TM_COLS);
         ptx::tmem_relinquish();
@@ -151,15 +178,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                                : 0u;
 
     const int n_items = p.batch * p.H;
-    const int G = gridDim.x;
-    // heads of this CTA: blockIdx.x + k * G; warps take the next k from a shared
-    // counter as they finish, so a warp held up by a merge head takes fewer heads
+    const int G = gridDim.x, bx = blockIdx.x;
+    const int kc = bx < n_items ? (n_items - 1 - bx) / G + 1 : 0;  // heads of this CTA
+    // with no more heads than warps every warp has one head and the order is moot
+    const bool pre = kc > NW && kc <= KMAX;
+    auto merges = [&](int s, int c) {
+        return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && c >= p.L - 1));
+    };
+    if (pre) {
+        for (int k = threadIdx.x; k < kc; k += NTHREADS) {
+            const int s = p.slots[(bx + k * G) / p.H];
+            const int c = (s >= 0 && s < p.n_slots && p.log_len) ? p.log_len[(size_t)s * p.n_layers + p.layer] : 0;
+            pre_slot[k] = s;
+            pre_len[k] = c;
+            if (merges(s, c)) atomicAdd(&cnt[0], 1);
+        }
+        __syncthreads();
+        const int nm = cnt[0];
+        for (int k = threadIdx.x; k < kc; k += NTHREADS) {
+            const int pos = merges(pre_slot[k], pre_len[k]) ? atomicAdd(&cnt[1], 1) : nm + atomicAdd(&cnt[2], 1);
+            order[pos] = (uint16_t)k;
+        }
+        __syncthreads();
+    }
+    auto item_at = [&](int pos) -> int {
+        if (pos >= kc) return n_items;
+        return bx + (pre ? (int)order[pos] : pos) * G;
+    };
+    // warps take the next position from a shared counter as they finish, so a warp
+    // held up by a merge head takes fewer heads
     auto grab = [&]() -> int {
-        int k = 0;
-        if (lane == 0) k = atomicAdd(next_k, 1);
-        k = __shfl_sync(FULL, k, 0);
-        const long long it = (long long)blockIdx.x + (long long)k * G;
-        return it < n_items ? (int)it : n_items;
+        int pos = 0;
+        if (lane == 0) pos = atomicAdd(next_k, 1);
+        return item_at(__shfl_sync(FULL, pos, 0));
     };
     const int E = p.E;
     const uint64_t pol_stream = ptx::policy_evict_first();
@@ -167,9 +218,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
     // -- head metadata: slot id first (it locates the tile and the log), live
     //    length after (it sizes the log part of the stream and decides the merge)
-    auto slot_of = [&](int it) -> int { return it < n_items ? p.slots[it / p.H] : -1; };
+    auto slot_of = [&](int it) -> int {
+        if (it >= n_items) return -1;
+        return pre ? pre_slot[(it - bx) / G] : p.slots[it / p.H];
+    };
     auto len_of = [&](const Head &hd) -> int {
-        return (hd.ok && p.log_len) ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
+        if (!hd.ok) return 0;
+        if (pre) return pre_len[(hd.it - bx) / G];
+        return p.log_len ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
     };
     auto resolve_slot = [&](Head &hd, int it, int s) {
         hd.it = it;
@@ -222,7 +278,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     Head cur, nxt;
     nxt.ok = 0;
     nxt.n = 0;
-    const int it0 = (long long)blockIdx.x + (long long)w * G < n_items ? blockIdx.x + w * G : n_items;
+    const int it0 = item_at(w);
     warm_token(it0);
     resolve_slot(cur, it0, slot_of(it0));
     int it_nxt = grab();                 // the warp's next head, and its slot id, one head early
@@ -363,6 +419,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                 kq = fmaf(q_own[x], k_own[x], kq);
             }
             kq = warp_allsum(kq);
+            // row vectors for the row blocks' broadcasts
+            reinterpret_cast<float4 *>(rv_qt)[lane] = make_float4(qt[0], qt[1], qt[2], qt[3]);
+            if (DELTA) reinterpret_cast<float4 *>(rv_kt)[lane] = make_float4(kt[0], kt[1], kt[2], kt[3]);
+            reinterpret_cast<float4 *>(rv_e)[lane] = make_float4(e_own[0], e_own[1], e_own[2], e_own[3]);
+            reinterpret_cast<float4 *>(rv_k)[lane] = make_float4(k_own[0], k_own[1], k_own[2], k_own[3]);
+            reinterpret_cast<float4 *>(rv_l)[lane] = make_float4(ell[0], ell[1], ell[2], ell[3]);
+            __syncwarp();
 
             // -- ReplayPrep + value replay over the log chunks (newest first):
             //    Y += (q^T A'_i) b_i, (k^T A'_i) b_i; a merge also stages A'_i, b_i in TMEM
@@ -431,28 +494,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (stage_tm) ptx::tmem_wait_st();
 
             // new rows of one 16-row block of the merged state from its Sbar rows in
-            // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending
+            // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending.
+            // A'_i rows of the block are published AG entries at a time by the block's
+            // four owner lanes and read by every lane as broadcasts.
             auto write_rows = [&](const float *sb, int cx, const float4 &bt4) {
                 float4 acc[CR];
 #pragma unroll
-                for (int rr = 0; rr < CR; ++rr) {
-                    const float4 S = reinterpret_cast<const float4 *>(sb + rr * DV)[lane];
-                    const float e = __shfl_sync(FULL, e_own[rr & 3], 4 * cx + (rr >> 2));
-                    acc[rr] = make_float4(S.x * e, S.y * e, S.z * e, S.w * e);
+                for (int r4 = 0; r4 < CR / 4; ++r4) {
+                    const float4 e4 = reinterpret_cast<const float4 *>(rv_e + cx * CR)[r4];
+                    const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const float4 S = reinterpret_cast<const float4 *>(sb + (4 * r4 + y) * DV)[lane];
+                        acc[4 * r4 + y] = make_float4(S.x * ev[y], S.y * ev[y], S.z * ev[y], S.w * ev[y]);
+                    }
                 }
                 const int nj = stage_tm ? c : 0;  // TMEM is read only where it was written
-                for (int j = 0; j < nj; ++j) {
-                    float tv[8];
-                    ptx::tmem_ld8(tm + 8u * (uint32_t)j, tv);
-                    const float4 b4 = make_float4(tv[4], tv[5], tv[6], tv[7]);
+                for (int j0 = 0; j0 < nj; j0 += AG) {
+                    float tv[8 * AG];
+                    ptx::tmem_ld32(tm + 8u * (uint32_t)j0, tv);
+                    if ((lane >> 2) == cx) {
 #pragma unroll
-                    for (int rr = 0; rr < CR; ++rr)
-                        fma4(acc[rr], __shfl_sync(FULL, tv[rr & 3], 4 * cx + (rr >> 2)), b4);
+                        for (int g = 0; g < AG; ++g)
+                            reinterpret_cast<float4 *>(ag + g * CR)[lane & 3] =
+                                make_float4(tv[8 * g], tv[8 * g + 1], tv[8 * g + 2], tv[8 * g + 3]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int g = 0; g < AG; ++g) {
+                        if (j0 + g < nj) {
+                            const float4 b4 = make_float4(tv[8 * g + 4], tv[8 * g + 5], tv[8 * g + 6], tv[8 * g + 7]);
+#pragma unroll
+                            for (int r4 = 0; r4 < CR / 4; ++r4) {
+                                const float4 a4 = reinterpret_cast<const float4 *>(ag + g * CR)[r4];
+                                fma4(acc[4 * r4 + 0], a4.x, b4);
+                                fma4(acc[4 * r4 + 1], a4.y, b4);
+                                fma4(acc[4 * r4 + 2], a4.z, b4);
+                                fma4(acc[4 * r4 + 3], a4.w, b4);
+                            }
+                        }
+                    }
+                    __syncwarp();
                 }
 #pragma unroll
-                for (int rr = 0; rr < CR; ++rr) {
-                    fma4(acc[rr], __shfl_sync(FULL, k_own[rr & 3], 4 * cx + (rr >> 2)), bt4);
-                    __stcs(reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane, acc[rr]);
+                for (int r4 = 0; r4 < CR / 4; ++r4) {
+                    const float4 k4 = reinterpret_cast<const float4 *>(rv_k + cx * CR)[r4];
+                    const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const int rr = 4 * r4 + y;
+                        fma4(acc[rr], kv[y], bt4);
+                        __stcs(reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane, acc[rr]);
+                    }
                 }
             };
 
@@ -463,11 +556,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                 if (!wait_chunk()) { abort = true; break; }
                 const float *sb = st + (size_t)(gc % NSW) * CF;
 #pragma unroll
-                for (int rr = 0; rr < CR; ++rr) {
-                    const float4 S = reinterpret_cast<const float4 *>(sb + rr * DV)[lane];
-                    const int src = 4 * cx + (rr >> 2);
-                    fma4(Yq, __shfl_sync(FULL, qt[rr & 3], src), S);
-                    if (DELTA) fma4(Yk, __shfl_sync(FULL, kt[rr & 3], src), S);
+                for (int r4 = 0; r4 < CR / 4; ++r4) {
+                    const float4 q4 = reinterpret_cast<const float4 *>(rv_qt + cx * CR)[r4];
+                    const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+                    float kv[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (DELTA) {
+                        const float4 k4 = reinterpret_cast<const float4 *>(rv_kt + cx * CR)[r4];
+                        kv[0] = k4.x; kv[1] = k4.y; kv[2] = k4.z; kv[3] = k4.w;
+                    }
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const float4 S = reinterpret_cast<const float4 *>(sb + (4 * r4 + y) * DV)[lane];
+                        fma4(Yq, qv[y], S);
+                        if (DELTA) fma4(Yk, kv[y], S);
+                    }
                 }
                 if (!DELTA && mk == MK_FUSED) write_rows(sb, cx, v4);
                 release();
@@ -490,10 +592,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (mk == MK_APPEND) {
                 float *ent = ring + (size_t)c * E;
                 *reinterpret_cast<float4 *>(ent + DK + 4 * lane) = bt4;
-                *reinterpret_cast<float4 *>(ent + 4 * lane) = make_float4(k_own[0], k_own[1], k_own[2], k_own[3]);
+                *reinterpret_cast<float4 *>(ent + 4 * lane) = reinterpret_cast<const float4 *>(rv_k)[lane];
                 if (DECAY == DL_DECAY_DIAG)
-                    *reinterpret_cast<float4 *>(ent + DK + DV + 4 * lane) = make_float4(ell[0], ell[1], ell[2], ell[3]);
-                if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[DK + DV] = ell[0];
+                    *reinterpret_cast<float4 *>(ent + DK + DV + 4 * lane) = reinterpret_cast<const float4 *>(rv_l)[lane];
+                if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[DK + DV] = rv_l[0];
             } else if (mk == MK_PASS2) {
                 // -- pass 2: the tile again (from L2), rewritten row block by row block
                 for (int cx = 0; cx < NCH; ++cx) {
@@ -547,16 +649,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                             if (i >= g1) continue;
                             float4 aw, bw;
                             if (i < c) {
+                                const float4 l4 = reinterpret_cast<const float4 *>(rv_l)[lane];
+                                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
                                 const float av[4] = {A[u].x, A[u].y, A[u].z, A[u].w};
                                 const float Lv[4] = {Lq[u].x, Lq[u].y, Lq[u].z, Lq[u].w};
                                 float w4[4];
 #pragma unroll
                                 for (int x = 0; x < 4; ++x)
-                                    w4[x] = DECAY == DL_DECAY_NONE ? av[x] : av[x] * expf(ell[x] - Lv[x]);
+                                    w4[x] = DECAY == DL_DECAY_NONE ? av[x] : av[x] * expf(lv[x] - Lv[x]);
                                 aw = make_float4(w4[0], w4[1], w4[2], w4[3]);
                                 bw = B[u];
                             } else {
-                                aw = make_float4(k_own[0], k_own[1], k_own[2], k_own[3]);
+                                aw = reinterpret_cast<const float4 *>(rv_k)[lane];
                                 bw = bt4;
                             }
                             reinterpret_cast<float4 *>(As + (size_t)(i - g0) * DK)[lane] = aw;
@@ -576,7 +680,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                         for (int rr = 0; rr < CR; ++rr) {
                             const float4 S = reinterpret_cast<const float4 *>(sb + rr * DV)[lane];
                             if (first) {
-                                const float e = __shfl_sync(FULL, e_own[rr & 3], 4 * cx + (rr >> 2));
+                                const float e = rv_e[cx * CR + rr];
                                 acc[rr] = make_float4(S.x * e, S.y * e, S.z * e, S.w * e);
                             } else {
                                 acc[rr] = S;
