@@ -128,8 +128,9 @@ def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph"):
 def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str) -> str:
     """Text for profiles/step_kernel_traffic.txt from an ncu --csv export of
     dram__bytes_read.sum and dram__bytes_write.sum over consecutive launches of the
-    hot kernel (one full merge interval, so the mix of append and merge launches
-    matches the timed region).  Run: python bench.py --traffic-from <csv>."""
+    hot kernel (a whole merge cycle of every slot group: rotation groups x log
+    capacity launches, so the mix of append and merge launches matches the timed
+    region).  Run: python bench.py --traffic-from <csv>."""
     import csv
     import re
     rows = list(csv.reader(open(csv_path)))
@@ -153,7 +154,8 @@ def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str
         raise SystemExit("no matching launches in " + csv_path)
     avg = sum(vals) / len(vals)
     return (f"# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the hot kernel,\n"
-            f"# averaged over {len(vals)} consecutive launches (one merge interval).\n"
+            f"# averaged over {len(vals)} consecutive launches (a whole merge cycle of every\n"
+            f"# slot group, so append and merge launches mix as in the timed region).\n"
             f"workload = {workload_key}\nkernel_sha = {kernel_source_hash()}\n"
             f"launches = {len(vals)}\ndram_bytes_per_launch = {avg:.0f}\n"
             f"min_launch_bytes = {min(vals):.0f}\nmax_launch_bytes = {max(vals):.0f}\n")
