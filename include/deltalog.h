@@ -77,6 +77,22 @@ typedef enum {
 
 typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
 
+/* Log entry layout.  The deferred log is that of the Design section; the narrower
+ * factor storage follows the per-operator instantiations of Section 3.4, which keep
+ * a_t in 16-bit storage (GDN, KDA), b_t in FP32 under the delta rule and both
+ * factors in BF16 for RWKV6, with the decay metadata in FP32.
+ *  DL_LOG_FP32     [a_i | b_i | Lambda_i] in fp32, 2*d_k + d_v floats per entry.
+ *  DL_LOG_COMPACT  [a_i bf16 x d_k | b_i | Lambda_i], where b_i is bf16 x d_v under
+ *                  DL_UPDATE_ADD and fp32 x d_v under the delta rule, and Lambda_i is
+ *                  fp32 x d_k (per-key decay), fp32 x 4 (scalar decay: Lambda_0 and 3
+ *                  pad floats) or absent (no decay).  a_t = k_t and, without the delta
+ *                  rule, b_t = v_t are bf16 inputs, so the narrower storage is exact:
+ *                  a compact pool computes the same values as an fp32 one while moving
+ *                  17-50% fewer log bytes.  Decode and append steps on a compact pool
+ *                  require in_dtype == DL_BF16 (else DL_ERR_DTYPE).
+ * dl_log_bytes gives the size of the log buffer either layout needs. */
+typedef enum { DL_LOG_FP32 = 0, DL_LOG_COMPACT = 1 } dl_log_format;
+
 /* Sticky device error bits (dl_read_error). */
 #define DL_EBIT_SLOT_RANGE 0x1  /* a slot id outside [0, n_slots)                    */
 #define DL_EBIT_LOG_FULL 0x2    /* append / decode without auto-merge on a full log   */
@@ -94,11 +110,12 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
  *
  *  state    [n_slots][n_layers][n_heads][d_k][d_v]  fp32 dense base state.  The
  *           caller writes prefill states here, then resets the slot's log.
- *  log      [n_slots][n_layers][n_heads][log_cap][2*d_k + d_v] fp32 ring.  Row i
- *           holds entry i as [a_i (d_k) | b_i (d_v) | Lambda_i (d_k)]; scalar decay
- *           uses Lambda_i[0] only; no decay leaves Lambda unused.  NULL makes an
- *           eager-only pool (decode/append/merge/materialize then return
- *           DL_ERR_UNSUPPORTED).
+ *  log      [n_slots][n_layers][n_heads][log_cap][entry] ring, 16-byte aligned.  Row i
+ *           holds entry i.  With log_format DL_LOG_FP32 an entry is
+ *           [a_i (d_k) | b_i (d_v) | Lambda_i (d_k)] fp32; scalar decay uses
+ *           Lambda_i[0] only; no decay leaves Lambda unused.  DL_LOG_COMPACT is
+ *           described at dl_log_format.  NULL makes an eager-only pool
+ *           (decode/append/merge/materialize then return DL_ERR_UNSUPPORTED).
  *  log_len  [n_slots][n_layers] int32 live-log length (entries 0..log_len-1 live).
  *           Required with a log; optional (NULL) for an eager-only pool.
  *  arrive   [n_slots][n_layers] int32 arrival counters used to commit log_len once
@@ -114,6 +131,7 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
  *           hold and there are at least as many heads as SMs, else 32 columns
  *           unless that leaves SMs idle, else 16).  32 needs d_k >= 64 and d_v a
  *           multiple of 32.
+ *  log_format dl_log_format of the log (DL_LOG_FP32 or DL_LOG_COMPACT).
  *
  * The cumulative log-decay lbar of a slot is not stored separately: it equals
  * Lambda of the newest live entry (0 when the log is empty).
@@ -123,6 +141,7 @@ typedef struct {
     dl_decay decay;
     dl_update update;
     int32_t tile_v;
+    int32_t log_format;  /* dl_log_format */
     float *state;
     float *log;
     int32_t *log_len;
@@ -155,6 +174,12 @@ typedef struct {
     const float *beta;
     float *out;
 } dl_step_args;
+
+/* Bytes of the log buffer a descriptor needs: n_slots * n_layers * n_heads *
+ * log_cap entries of the layout its log_format, decay and update select (every
+ * entry a multiple of 16 bytes).  Reads only the shape fields and log_format;
+ * DL_ERR_SHAPE / DL_ERR_INVALID_ARG as dl_create_pool for those.  No CUDA call. */
+dl_status dl_log_bytes(const dl_pool_desc *desc, int64_t *bytes);
 
 /* Validate a descriptor and return a host handle recording it.  No device
  * memory is allocated and no CUDA call is made. */

@@ -22,6 +22,27 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool dk_supported(int dk) { return dk == 16 || dk == 64 || dk == 128; }
 
+// Log entry layout of a descriptor (dl_log_format in deltalog.h), in floats.
+struct LogLayout {
+    int E, boff, loff, a16, b16;
+};
+LogLayout log_layout(const dl_pool_desc &d) {
+    LogLayout l;
+    if (d.log_format == DL_LOG_COMPACT) {
+        l.a16 = 1;
+        l.b16 = d.update == DL_UPDATE_ADD ? 1 : 0;
+        l.boff = d.d_k / 2;
+        l.loff = l.boff + (l.b16 ? d.d_v / 2 : d.d_v);
+        l.E = l.loff + (d.decay == DL_DECAY_DIAG ? d.d_k : d.decay == DL_DECAY_SCALAR ? 4 : 0);
+    } else {
+        l.a16 = l.b16 = 0;
+        l.boff = d.d_k;
+        l.loff = d.d_k + d.d_v;
+        l.E = 2 * d.d_k + d.d_v;
+    }
+    return l;
+}
+
 dl::KParams base_params(const dl_pool_desc &d, int layer) {
     dl::KParams p;
     std::memset(&p, 0, sizeof(p));
@@ -37,7 +58,12 @@ dl::KParams base_params(const dl_pool_desc &d, int layer) {
     p.dk = d.d_k;
     p.dv = d.d_v;
     p.L = d.log_cap;
-    p.E = 2 * d.d_k + d.d_v;
+    const LogLayout l = log_layout(d);
+    p.E = l.E;
+    p.boff = l.boff;
+    p.loff = l.loff;
+    p.a16 = l.a16;
+    p.b16 = l.b16;
     p.layer = layer;
     return p;
 }
@@ -65,7 +91,8 @@ bool use_whole_head(const dl_pool_desc &d, const dl_step_args *a, bool want_out,
     return (long long)a->batch * d.n_heads >= (long long)dl::device_sm_count();
 }
 
-dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, bool need_out) {
+dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, bool need_out,
+                     bool uses_log) {
     if (!P || !a) return DL_ERR_INVALID_ARG;
     const dl_pool_desc &d = P->d;
     if (layer < 0 || layer >= d.n_layers) return DL_ERR_INVALID_ARG;
@@ -74,6 +101,8 @@ dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, boo
     if (a->batch > d.n_slots) return DL_ERR_SHAPE;
     if (!a->slots || !a->q || !a->k || !a->v) return DL_ERR_INVALID_ARG;
     if (a->in_dtype != DL_F32 && a->in_dtype != DL_BF16) return DL_ERR_DTYPE;
+    // the compact log stores a_t = k_t (and b_t = v_t) in bf16: exact only for bf16 inputs
+    if (uses_log && d.log_format == DL_LOG_COMPACT && a->in_dtype != DL_BF16) return DL_ERR_DTYPE;
     const uintptr_t esz = a->in_dtype == DL_F32 ? 4 : 2;
     if (!aligned(a->q, esz) || !aligned(a->k, esz) || !aligned(a->v, esz)) return DL_ERR_INVALID_ARG;
     if (d.decay != DL_DECAY_NONE && (!a->lambda || !aligned(a->lambda, 4))) return DL_ERR_INVALID_ARG;
@@ -117,6 +146,20 @@ dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_o
 
 }  // namespace
 
+DL_API dl_status dl_log_bytes(const dl_pool_desc *desc, int64_t *bytes) {
+    if (!desc || !bytes) return DL_ERR_INVALID_ARG;
+    const dl_pool_desc &d = *desc;
+    if (d.n_slots <= 0 || d.n_layers <= 0 || d.n_heads <= 0) return DL_ERR_SHAPE;
+    if (!dk_supported(d.d_k) || d.d_v < 16 || d.d_v > 1024 || d.d_v % 16) return DL_ERR_SHAPE;
+    if (d.log_cap < 1 || d.log_cap > 64) return DL_ERR_SHAPE;
+    if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
+    if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
+        return DL_ERR_INVALID_ARG;
+    if (d.log_format != DL_LOG_FP32 && d.log_format != DL_LOG_COMPACT) return DL_ERR_INVALID_ARG;
+    *bytes = (int64_t)d.n_slots * d.n_layers * d.n_heads * d.log_cap * log_layout(d).E * 4;
+    return DL_OK;
+}
+
 DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
     if (!desc || !out_pool) return DL_ERR_INVALID_ARG;
     *out_pool = nullptr;
@@ -133,6 +176,7 @@ DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
     if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;
+    if (d.log_format != DL_LOG_FP32 && d.log_format != DL_LOG_COMPACT) return DL_ERR_INVALID_ARG;
     if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
         return DL_ERR_INVALID_ARG;
     if (d.log && (!aligned(d.log, 16) || !d.log_len || !d.arrive)) return DL_ERR_INVALID_ARG;
@@ -155,14 +199,14 @@ DL_API dl_status dl_destroy_pool(dl_pool *pool) {
 
 DL_API dl_status dl_decode_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
                                 int32_t auto_merge, void *stream) {
-    const dl_status s = check_step(pool, layer, args, true);
+    const dl_status s = check_step(pool, layer, args, true, true);
     if (s != DL_OK || args->batch == 0) return s;
     if (!pool->d.log) return DL_ERR_UNSUPPORTED;
     return run_step(pool, layer, args, true, auto_merge != 0, false, stream);
 }
 
 DL_API dl_status dl_append(dl_pool *pool, int32_t layer, const dl_step_args *args, void *stream) {
-    const dl_status s = check_step(pool, layer, args, false);
+    const dl_status s = check_step(pool, layer, args, false, true);
     if (s != DL_OK || args->batch == 0) return s;
     if (!pool->d.log) return DL_ERR_UNSUPPORTED;
     return run_step(pool, layer, args, false, false, false, stream);
@@ -170,7 +214,7 @@ DL_API dl_status dl_append(dl_pool *pool, int32_t layer, const dl_step_args *arg
 
 DL_API dl_status dl_eager_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
                                void *stream) {
-    const dl_status s = check_step(pool, layer, args, true);
+    const dl_status s = check_step(pool, layer, args, true, false);
     if (s != DL_OK || args->batch == 0) return s;
     return run_step(pool, layer, args, true, false, true, stream);
 }
@@ -268,12 +312,20 @@ dl_status check_desc_without_arrive(const dl_pool_desc &d) {
     if ((int)d.decay < DL_DECAY_NONE || (int)d.decay > DL_DECAY_DIAG) return DL_ERR_INVALID_ARG;
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;
+    if (d.log_format != DL_LOG_FP32 && d.log_format != DL_LOG_COMPACT) return DL_ERR_INVALID_ARG;
     if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
         return DL_ERR_INVALID_ARG;
     if (!d.log || !aligned(d.log, 16) || !d.log_len || !aligned(d.log_len, 4))
         return DL_ERR_INVALID_ARG;
     if ((long long)d.n_slots * d.n_heads * (d.d_v / 16) > 0x7fffffffLL) return DL_ERR_SHAPE;
     return DL_OK;
+}
+
+// The host-side checks of dl_decode_step for a descriptor (no CUDA call).
+dl_status check_decode_args(const dl_pool_desc &desc, int32_t layer, const dl_step_args *args) {
+    dl_pool stack_pool;
+    stack_pool.d = desc;
+    return check_step(&stack_pool, layer, args, true, true);
 }
 
 // Runs dl_decode_step for a checked descriptor with the given arrival counters,

@@ -19,7 +19,11 @@ struct KParams {
     int32_t *arrive;
     int32_t *err;
     int n_slots, n_layers, H, Hk, dk, dv, L;
-    int E;      // floats per log entry: 2*d_k + d_v
+    int E;      // floats per log entry (the layout's entry bytes / 4)
+    int boff;   // offset of b_i in an entry, in floats
+    int loff;   // offset of Lambda_i in an entry, in floats
+    int a16;    // a_i stored as bf16 (compact layout)
+    int b16;    // b_i stored as bf16 (compact layout without the delta rule)
     int nv;     // value tiles per head: d_v / B_V
     int layer;
     // batch

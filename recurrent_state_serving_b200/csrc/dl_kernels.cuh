@@ -43,6 +43,38 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// ---- log entry access.  The layout (fp32, or compact with bf16 a_i and, without the
+// delta rule, bf16 b_i) comes from KParams; Lambda_i is fp32 at p.loff either way.
+__device__ __forceinline__ float4 bf16x4_to_float4(const __nv_bfloat16 *src) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+    return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+// a_i[4 r4 .. 4 r4 + 3]
+__device__ __forceinline__ float4 ent_a4(const KParams &p, const float *ent, int r4) {
+    if (p.a16) return bf16x4_to_float4(reinterpret_cast<const __nv_bfloat16 *>(ent) + 4 * r4);
+    return *reinterpret_cast<const float4 *>(ent + 4 * r4);
+}
+// b_i[4 c4 .. 4 c4 + 3]
+__device__ __forceinline__ float4 ent_b4(const KParams &p, const float *ent, int c4) {
+    if (p.b16) return bf16x4_to_float4(reinterpret_cast<const __nv_bfloat16 *>(ent + p.boff) + 4 * c4);
+    return *reinterpret_cast<const float4 *>(ent + p.boff + 4 * c4);
+}
+__device__ __forceinline__ float ent_a(const KParams &p, const float *ent, int r) {
+    return p.a16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(ent)[r]) : ent[r];
+}
+// the stored values are bf16 inputs (k_t, and v_t without the delta rule), so the
+// conversion back to bf16 is exact
+__device__ __forceinline__ void ent_put_a(const KParams &p, float *ent, int r, float v) {
+    if (p.a16) reinterpret_cast<__nv_bfloat16 *>(ent)[r] = __float2bfloat16_rn(v);
+    else ent[r] = v;
+}
+__device__ __forceinline__ void ent_put_b(const KParams &p, float *ent, int col, float v) {
+    if (p.b16) reinterpret_cast<__nv_bfloat16 *>(ent + p.boff)[col] = __float2bfloat16_rn(v);
+    else ent[p.boff + col] = v;
+}
+
 __device__ __forceinline__ void fma4(float4 &acc, float a, const float4 &b) {
     acc.x = fmaf(a, b.x, acc.x);
     acc.y = fmaf(a, b.y, acc.y);
@@ -141,7 +173,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     const int g = h / (p.H / p.Hk);
     const IT *qrow = static_cast<const IT *>(p.q) + ((size_t)bi * p.Hk + g) * DK;
     const IT *krow = static_cast<const IT *>(p.k) + ((size_t)bi * p.Hk + g) * DK;
-    const float *Lprev = (c > 0) ? ring + (size_t)(c - 1) * p.E + DK + dv : nullptr;
+    const float *Lprev = (c > 0) ? ring + (size_t)(c - 1) * p.E + p.loff : nullptr;
     float lam_s = 0.f;
     const float *lrow = nullptr;
     if (DECAY == DL_DECAY_SCALAR) lam_s = p.lam_const ? p.lam[h] : p.lam[(size_t)bi * p.H + h];
@@ -176,15 +208,15 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         const float *ent = ring + (size_t)i * p.E;
         float fs = 1.f, fk = 1.f;
         if (DECAY == DL_DECAY_SCALAR) {
-            const float Li = ent[DK + dv];
+            const float Li = ent[p.loff];
             fs = expf(s_ell[0] - Li);
             fk = (DELTA && p.undecayed) ? expf(s_ellp[0] - Li) : fs;
         }
         float pq = 0.f, pk = 0.f;
         for (int r4 = lane; r4 < DK / 4; r4 += 32) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(ent + 4 * r4);
+            const float4 a4 = ent_a4(p, ent, r4);
             float4 L4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (DECAY == DL_DECAY_DIAG) L4 = *reinterpret_cast<const float4 *>(ent + DK + dv + 4 * r4);
+            if (DECAY == DL_DECAY_DIAG) L4 = *reinterpret_cast<const float4 *>(ent + p.loff + 4 * r4);
             const float av[4] = {a4.x, a4.y, a4.z, a4.w};
             const float Lv[4] = {L4.x, L4.y, L4.z, L4.w};
 #pragma unroll
@@ -213,8 +245,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     // value-side log shard of this tile
     for (int idx = tid; idx < c * CQ; idx += NT) {
         const int i = idx / CQ, x4 = idx % CQ;
-        reinterpret_cast<float4 *>(s_b + i * BV)[x4] =
-            *reinterpret_cast<const float4 *>(ring + (size_t)i * p.E + DK + (size_t)j * BV + 4 * x4);
+        reinterpret_cast<float4 *>(s_b + i * BV)[x4] = ent_b4(p, ring + (size_t)i * p.E, (j * BV) / 4 + x4);
     }
     if (p.want_out && warp == 0) {  // a_t . q_t for the new entry (no decay since insertion)
         float x = 0.f;
@@ -281,16 +312,16 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         const float vv = to_f32(static_cast<const IT *>(p.v)[row * dv + col]);
         const float bt = DELTA ? p.beta[row] * (vv - Yk) : vv;
         if (p.want_out) p.out[row * dv + col] = fmaf(bt, s_kq, Yq);
-        if (!merge_now) ring[(size_t)c * p.E + DK + col] = bt;
+        if (!merge_now) ent_put_b(p, ring + (size_t)c * p.E, col, bt);
         s_bt[tid] = bt;
     }
     if (!merge_now && j == 0) {  // designated writer of the shared entry fields
         float *ent = ring + (size_t)c * p.E;
         for (int r = tid; r < DK; r += NT) {
-            ent[r] = s_k[r];
-            if (DECAY == DL_DECAY_DIAG) ent[DK + dv + r] = s_ell[r];
+            ent_put_a(p, ent, r, s_k[r]);
+            if (DECAY == DL_DECAY_DIAG) ent[p.loff + r] = s_ell[r];
         }
-        if (DECAY == DL_DECAY_SCALAR && tid == 0) ent[DK + dv] = s_ell[0];
+        if (DECAY == DL_DECAY_SCALAR && tid == 0) ent[p.loff] = s_ell[0];
     }
 
     // 7. merge step: write the materialised state back over the base tile
@@ -379,7 +410,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     const float *ring = p.log + head * (size_t)p.L * p.E;
     const DynLayout lay(p.L, BV);
     float *s_b = s_dyn + lay.b, *s_A = s_dyn + lay.A;
-    const float *Lbar = (c > 0) ? ring + (size_t)(c - 1) * p.E + DK + dv : nullptr;
+    const float *Lbar = (c > 0) ? ring + (size_t)(c - 1) * p.E + p.loff : nullptr;
 
     for (int r = tid; r < DK; r += NT) {
         float e = 1.f;
@@ -390,15 +421,14 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     for (int idx = tid; idx < c * DK; idx += NT) {
         const int i = idx / DK, r = idx % DK;
         const float *ent = ring + (size_t)i * p.E;
-        float w = ent[r];
-        if (DECAY == DL_DECAY_DIAG) w *= expf(Lbar[r] - ent[DK + dv + r]);
-        if (DECAY == DL_DECAY_SCALAR) w *= expf(Lbar[0] - ent[DK + dv]);
+        float w = ent_a(p, ent, r);
+        if (DECAY == DL_DECAY_DIAG) w *= expf(Lbar[r] - ent[p.loff + r]);
+        if (DECAY == DL_DECAY_SCALAR) w *= expf(Lbar[0] - ent[p.loff]);
         s_A[idx] = w;
     }
     for (int idx = tid; idx < c * CQ; idx += NT) {
         const int i = idx / CQ, x4 = idx % CQ;
-        reinterpret_cast<float4 *>(s_b + i * BV)[x4] =
-            *reinterpret_cast<const float4 *>(ring + (size_t)i * p.E + DK + (size_t)j * BV + 4 * x4);
+        reinterpret_cast<float4 *>(s_b + i * BV)[x4] = ent_b4(p, ring + (size_t)i * p.E, (j * BV) / 4 + x4);
     }
     __syncthreads();
 

@@ -82,16 +82,23 @@ static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and s
 static_assert(TM_ENT * 8 <= (int)TM_WCOLS, "A'_i and b_i take 8 columns per entry");
 constexpr unsigned FULL = 0xffffffffu;
 
-// A log entry as copied into shared memory: [a | b | Lambda] for per-key decay
-// (the whole ring row), [a | b | Lambda_0 and 3 pad floats] for scalar decay,
-// [a | b] without decay.  EPC entries fill one stage.
-template <int DECAY>
+// Log entry layout (FMT 0: fp32 [a | b | Lambda]; FMT 1: compact, a bf16, b bf16 without
+// the delta rule, Lambda fp32 x d_k / x 4 / absent) and how entries travel through a
+// stage.  Whole ring rows are copied when they hold nothing unused (compact rows, or
+// per-key decay); otherwise each entry's [a | b | Lambda_0 and 3 pad floats] (scalar
+// decay) or [a | b] (no decay) is copied.  Up to EPC entries fill one stage.
+template <int DECAY, int FMT, bool DELTA>
 struct LogCopy {
-    static constexpr uint32_t ESB = DECAY == DL_DECAY_DIAG     ? (2 * DK + DV) * 4
-                                    : DECAY == DL_DECAY_SCALAR ? (DK + DV + 4) * 4
-                                                               : (DK + DV) * 4;
+    static constexpr bool A16 = FMT == 1;
+    static constexpr bool B16 = FMT == 1 && !DELTA;
+    static constexpr int B_OFF = A16 ? DK / 2 : DK;            // b_i in floats from the row start
+    static constexpr int L_OFF = B_OFF + (B16 ? DV / 2 : DV);   // Lambda_i
+    static constexpr int E_F = FMT == 1 ? L_OFF + (DECAY == DL_DECAY_DIAG ? DK : DECAY == DL_DECAY_SCALAR ? 4 : 0)
+                                        : 2 * DK + DV;          // ring row in floats
+    static constexpr bool WHOLE = FMT == 1 || DECAY == DL_DECAY_DIAG;
+    static constexpr uint32_t ESB = WHOLE ? E_F * 4 : (L_OFF + (DECAY == DL_DECAY_SCALAR ? 4 : 0)) * 4;
     static constexpr int ESF = ESB / 4;
-    static constexpr int EPC = CB / ESB;
+    static constexpr int EPC = CB / ESB < 8 ? CB / ESB : 8;     // capped: the replay unrolls a stage
 };
 
 template <typename T> __device__ __forceinline__ void load4(const T *p, float (&v)[4]);
@@ -133,12 +140,38 @@ struct Head {
     size_t head;   // (slot, layer, head) index
 };
 
-template <int DECAY, bool DELTA, typename IT>
+// a_i[4l .. 4l + 3] or b_i[4l .. 4l + 3] of an entry (shared or global memory)
+template <bool HALF>
+__device__ __forceinline__ float4 seg4(const float *seg, int lane) {
+    if (HALF) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(seg) + 4 * lane);
+        const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(&u.x);
+        const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(&u.y);
+        return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+    }
+    return reinterpret_cast<const float4 *>(seg)[lane];
+}
+// the values stored narrow are bf16 inputs (k_t; v_t without the delta rule): exact
+template <bool HALF>
+__device__ __forceinline__ void put_seg4(float *seg, int lane, float4 v) {
+    if (HALF) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t *>(&lo);
+        u.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(seg) + 4 * lane) = u;
+    } else {
+        reinterpret_cast<float4 *>(seg)[lane] = v;
+    }
+}
+
+template <int DECAY, bool DELTA, typename IT, int FMT>
 __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 {
-    using LC = LogCopy<DECAY>;
+    using LC = LogCopy<DECAY, FMT, DELTA>;
     constexpr uint32_t ESB = LC::ESB;
     constexpr int ESF = LC::ESF, EPC = LC::EPC;
+    constexpr int BO = LC::B_OFF, LO = LC::L_OFF;
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -295,7 +328,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             const int hi = hd.c - EPC * x, lo = hi - EPC > 0 ? hi - EPC : 0;
             const float *src = p.log + hd.head * (size_t)p.L * E;
             ptx::mbar_arrive_expect_tx(bar, (uint32_t)(hi - lo) * ESB);
-            if (DECAY == DL_DECAY_DIAG) {
+            if (LC::WHOLE) {
                 ptx::bulk_g2s(dst, src + (size_t)lo * E, (uint32_t)(hi - lo) * ESB, bar, pol_stream);
             } else {
                 for (int i = lo; i < hi; ++i)
@@ -397,7 +430,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (c > 0) {
                 if (!wait_chunk()) { abort = true; break; }
                 const int lo0 = c - EPC > 0 ? c - EPC : 0;
-                const float *ent = st + (size_t)(gc % NSW) * CF + (size_t)(c - 1 - lo0) * ESF + DK + DV;
+                const float *ent = st + (size_t)(gc % NSW) * CF + (size_t)(c - 1 - lo0) * ESF + LO;
                 if (DECAY == DL_DECAY_DIAG) {
                     const float4 p4 = reinterpret_cast<const float4 *>(ent)[lane];
                     lp[0] = p4.x; lp[1] = p4.y; lp[2] = p4.z; lp[3] = p4.w;
@@ -441,13 +474,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     pk[e] = 0.f;
                     if (lo + e < hi) {
                         const float *ent = sb + (size_t)e * ESF;
-                        const float4 a4 = reinterpret_cast<const float4 *>(ent)[lane];
+                        const float4 a4 = seg4<LC::A16>(ent, lane);
                         float Lv[4] = {0.f, 0.f, 0.f, 0.f};
                         if (DECAY == DL_DECAY_DIAG) {
-                            const float4 L4 = reinterpret_cast<const float4 *>(ent + DK + DV)[lane];
+                            const float4 L4 = reinterpret_cast<const float4 *>(ent + LO)[lane];
                             Lv[0] = L4.x; Lv[1] = L4.y; Lv[2] = L4.z; Lv[3] = L4.w;
                         } else if (DECAY == DL_DECAY_SCALAR) {
-                            const float Ls = ent[DK + DV];
+                            const float Ls = ent[LO];
 #pragma unroll
                             for (int y = 0; y < 4; ++y) Lv[y] = Ls;
                         }
@@ -465,7 +498,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                             }
                         }
                         if (stage_tm) {
-                            const float4 b4 = reinterpret_cast<const float4 *>(ent + DK)[lane];
+                            const float4 b4 = seg4<LC::B16>(ent + BO, lane);
                             const float tv[8] = {wq[0], wq[1], wq[2], wq[3], b4.x, b4.y, b4.z, b4.w};
                             ptx::tmem_st8(tm + 8u * (uint32_t)(lo + e), tv);
                         }
@@ -483,7 +516,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 #pragma unroll
                 for (int e = 0; e < EPC; ++e) {
                     if (lo + e < hi) {
-                        const float4 b4 = reinterpret_cast<const float4 *>(sb + (size_t)e * ESF + DK)[lane];
+                        const float4 b4 = seg4<LC::B16>(sb + (size_t)e * ESF + BO, lane);
                         fma4(Yq, pq[e], b4);
                         if (DELTA) fma4(Yk, pk[e], b4);
                     }
@@ -591,11 +624,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                 *reinterpret_cast<float4 *>(p.out + row * DV + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
             if (mk == MK_APPEND) {
                 float *ent = ring + (size_t)c * E;
-                *reinterpret_cast<float4 *>(ent + DK + 4 * lane) = bt4;
-                *reinterpret_cast<float4 *>(ent + 4 * lane) = reinterpret_cast<const float4 *>(rv_k)[lane];
+                put_seg4<LC::B16>(ent + BO, lane, bt4);
+                put_seg4<LC::A16>(ent, lane, reinterpret_cast<const float4 *>(rv_k)[lane]);
                 if (DECAY == DL_DECAY_DIAG)
-                    *reinterpret_cast<float4 *>(ent + DK + DV + 4 * lane) = reinterpret_cast<const float4 *>(rv_l)[lane];
-                if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[DK + DV] = rv_l[0];
+                    *reinterpret_cast<float4 *>(ent + LO + 4 * lane) = reinterpret_cast<const float4 *>(rv_l)[lane];
+                if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[LO] = rv_l[0];
             } else if (mk == MK_PASS2) {
                 // -- pass 2: the tile again (from L2), rewritten row block by row block
                 for (int cx = 0; cx < NCH; ++cx) {
@@ -633,12 +666,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                             const int i = i0 + u;
                             if (i < g1 && i < c) {
                                 const float *ent = ring + (size_t)i * E;
-                                A[u] = ldg4(ent + 4 * lane);
-                                B[u] = ldg4(ent + DK + 4 * lane);
+                                A[u] = seg4<LC::A16>(ent, lane);
+                                B[u] = seg4<LC::B16>(ent + BO, lane);
                                 if (DECAY == DL_DECAY_DIAG) {
-                                    Lq[u] = ldg4(ent + DK + DV + 4 * lane);
+                                    Lq[u] = ldg4(ent + LO + 4 * lane);
                                 } else {
-                                    const float Ls = DECAY == DL_DECAY_SCALAR ? __ldg(ent + DK + DV) : 0.f;
+                                    const float Ls = DECAY == DL_DECAY_SCALAR ? __ldg(ent + LO) : 0.f;
                                     Lq[u] = make_float4(Ls, Ls, Ls, Ls);
                                 }
                             }

@@ -20,9 +20,14 @@ bool whole_head_supported(int dk, int dv) { return dk == wh::DK && dv == wh::DV;
 
 namespace {
 
-template <int DECAY, bool DELTA, typename IT>
+template <int DECAY, bool DELTA, typename IT, int FMT>
 cudaError_t launch_one(const KParams &p, cudaStream_t st) {
-    auto kern = wh::warp_head_kernel<DECAY, DELTA, IT>;
+    // the kernel's compile-time entry layout must be the one the pool was given
+    using LC = wh::LogCopy<DECAY, FMT, DELTA>;
+    if (p.log && (p.E != LC::E_F || p.boff != LC::B_OFF || p.loff != LC::L_OFF || p.a16 != (int)LC::A16 ||
+                  p.b16 != (int)LC::B16))
+        return cudaErrorInvalidValue;
+    auto kern = wh::warp_head_kernel<DECAY, DELTA, IT, FMT>;
     static bool configured = false;  // per instantiation
     if (!configured) {
         const cudaError_t e =
@@ -39,11 +44,16 @@ cudaError_t launch_one(const KParams &p, cudaStream_t st) {
 
 template <int DECAY>
 cudaError_t by_update(const KParams &p, bool delta, bool bf16, cudaStream_t st) {
+    if (p.a16) {  // compact log: bf16 inputs only (checked at the ABI)
+        if (!bf16) return cudaErrorInvalidValue;
+        return delta ? launch_one<DECAY, true, __nv_bfloat16, 1>(p, st)
+                     : launch_one<DECAY, false, __nv_bfloat16, 1>(p, st);
+    }
     if (delta)
-        return bf16 ? launch_one<DECAY, true, __nv_bfloat16>(p, st)
-                    : launch_one<DECAY, true, float>(p, st);
-    return bf16 ? launch_one<DECAY, false, __nv_bfloat16>(p, st)
-                : launch_one<DECAY, false, float>(p, st);
+        return bf16 ? launch_one<DECAY, true, __nv_bfloat16, 0>(p, st)
+                    : launch_one<DECAY, true, float, 0>(p, st);
+    return bf16 ? launch_one<DECAY, false, __nv_bfloat16, 0>(p, st)
+                : launch_one<DECAY, false, float, 0>(p, st);
 }
 
 }  // namespace

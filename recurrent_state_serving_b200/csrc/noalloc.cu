@@ -12,6 +12,7 @@
 
 namespace dl {
 dl_status check_desc_without_arrive(const dl_pool_desc &d);
+dl_status check_decode_args(const dl_pool_desc &desc, int32_t layer, const dl_step_args *args);
 dl_status decode_step_on_desc(const dl_pool_desc &desc, int32_t *arrive, int32_t layer,
                               const dl_step_args *args, int32_t auto_merge, void *stream);
 }
@@ -52,6 +53,9 @@ DL_API dl_status dl_decode_step_noalloc(const dl_pool_desc *desc, int32_t layer,
     if (v != DL_OK) return v;
     const long long counters = (long long)desc->n_slots * desc->n_layers;
     if (counters > DL_NOALLOC_MAX_COUNTERS) return DL_ERR_SHAPE;
+    // the step's own host-side checks come before any CUDA call
+    const dl_status a = dl::check_decode_args(*desc, layer, args);
+    if (a != DL_OK || args->batch == 0) return a;
     int32_t *scratch = nullptr;
     if (args->batch > 0) {
         const dl_status s = scratch_on_current_device(&scratch);

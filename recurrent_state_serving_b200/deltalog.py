@@ -29,6 +29,7 @@ DL_OK, DL_ERR_INVALID_ARG, DL_ERR_SHAPE, DL_ERR_DTYPE, DL_ERR_UNSUPPORTED, DL_ER
 DECAY = {"none": 0, "scalar": 1, "diag": 2}
 UPDATE = {"add": 0, "delta": 1, "delta_undecayed": 2}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+LOG_FORMAT = {"fp32": 0, "compact": 1}
 DL_EBIT_SLOT_RANGE, DL_EBIT_LOG_FULL, DL_EBIT_LIVE_LOG, DL_EBIT_LOG_LEN, DL_EBIT_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
 
@@ -38,7 +39,7 @@ class dl_pool_desc(ctypes.Structure):
                 ("n_heads", ctypes.c_int32), ("n_kheads", ctypes.c_int32),
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("log_cap", ctypes.c_int32),
                 ("decay", ctypes.c_int), ("update", ctypes.c_int), ("tile_v", ctypes.c_int32),
-                ("state", ctypes.c_void_p), ("log", ctypes.c_void_p),
+                ("log_format", ctypes.c_int32), ("state", ctypes.c_void_p), ("log", ctypes.c_void_p),
                 ("log_len", ctypes.c_void_p), ("arrive", ctypes.c_void_p),
                 ("err_word", ctypes.c_void_p)]
 
@@ -52,6 +53,7 @@ class dl_step_args(ctypes.Structure):
 
 
 _vp = ctypes.c_void_p
+_lib.dl_log_bytes.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.POINTER(ctypes.c_int64)]
 _lib.dl_create_pool.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.POINTER(_vp)]
 _lib.dl_destroy_pool.argtypes = [_vp]
 _lib.dl_decode_step.argtypes = [_vp, ctypes.c_int32, ctypes.POINTER(dl_step_args), ctypes.c_int32, _vp]
@@ -65,7 +67,7 @@ _lib.dl_decode_step_noalloc.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.c_i
                                         ctypes.POINTER(dl_step_args), ctypes.c_int32, _vp]
 _lib.dl_status_string.argtypes = [ctypes.c_int]
 _lib.dl_status_string.restype = ctypes.c_char_p
-for _f in ("dl_create_pool", "dl_destroy_pool", "dl_decode_step", "dl_append", "dl_eager_step",
+for _f in ("dl_log_bytes", "dl_create_pool", "dl_destroy_pool", "dl_decode_step", "dl_append", "dl_eager_step",
            "dl_merge", "dl_materialize", "dl_reset_slots", "dl_read_error", "dl_decode_step_noalloc"):
     getattr(_lib, _f).restype = ctypes.c_int
 
@@ -120,23 +122,30 @@ class Pool:
     """State pool + log ring + metadata in caller-owned (torch) device memory."""
 
     def __init__(self, n_slots, n_layers, n_heads, d_k, d_v, log_cap, decay="none",
-                 update="add", n_kheads=None, device="cuda", with_log=True, tile_v=0):
+                 update="add", n_kheads=None, device="cuda", with_log=True, tile_v=0,
+                 log_format="fp32"):
         dev = torch.device(device)
         n_kheads = n_heads if n_kheads is None else n_kheads
         self.n_slots, self.n_layers, self.n_heads, self.n_kheads = n_slots, n_layers, n_heads, n_kheads
         self.d_k, self.d_v, self.log_cap, self.decay, self.update = d_k, d_v, log_cap, decay, update
-        self.tile_v = tile_v
+        self.tile_v, self.log_format = tile_v, log_format
+        self.desc = dl_pool_desc(n_slots, n_layers, n_heads, n_kheads, d_k, d_v, log_cap,
+                                 DECAY[decay], UPDATE[update], tile_v, LOG_FORMAT[log_format])
+        nbytes = ctypes.c_int64()
+        _check(_lib.dl_log_bytes(ctypes.byref(self.desc), ctypes.byref(nbytes)), "dl_log_bytes")
+        # one entry in 4-byte words (its bf16 parts, if any, are packed in pairs)
+        self.entry_floats = nbytes.value // (4 * n_slots * n_layers * n_heads * log_cap)
         self.state = torch.zeros(n_slots, n_layers, n_heads, d_k, d_v, dtype=torch.float32, device=dev)
-        self.log = (torch.zeros(n_slots, n_layers, n_heads, log_cap, 2 * d_k + d_v,
+        self.log = (torch.zeros(n_slots, n_layers, n_heads, log_cap, self.entry_floats,
                                 dtype=torch.float32, device=dev) if with_log else None)
         self.log_len = torch.zeros(n_slots, n_layers, dtype=torch.int32, device=dev)
         self.arrive = torch.zeros(n_slots, n_layers, dtype=torch.int32, device=dev)
         self.err_word = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.desc = dl_pool_desc(n_slots, n_layers, n_heads, n_kheads, d_k, d_v, log_cap,
-                                 DECAY[decay], UPDATE[update], tile_v, self.state.data_ptr(),
-                                 None if self.log is None else self.log.data_ptr(),
-                                 self.log_len.data_ptr(), self.arrive.data_ptr(),
-                                 self.err_word.data_ptr())
+        self.desc.state = self.state.data_ptr()
+        self.desc.log = None if self.log is None else self.log.data_ptr()
+        self.desc.log_len = self.log_len.data_ptr()
+        self.desc.arrive = self.arrive.data_ptr()
+        self.desc.err_word = self.err_word.data_ptr()
         h = ctypes.c_void_p()
         _check(_lib.dl_create_pool(ctypes.byref(self.desc), ctypes.byref(h)), "dl_create_pool")
         self.handle = h
@@ -151,10 +160,6 @@ class Pool:
             self.close()
         except Exception:
             pass
-
-    @property
-    def entry_floats(self):
-        return 2 * self.d_k + self.d_v
 
 
 def _step_args(pool, slots, q, k, v, lam, beta, out, lambda_per_head):

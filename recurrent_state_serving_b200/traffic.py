@@ -12,7 +12,8 @@ replay reads and the periodic merge):
   standalone merge state read + write 8 d_k d_v + c log entries read
 
 A log entry is a_i (4 d_k) + b_i (4 d_v) + Lambda_i (4 d_k for per-key decay, 4 for
-scalar decay, 0 without decay).  Token I/O: q and k (shared by the n_heads/n_kheads
+scalar decay, 0 without decay).  In the compact layout a_i takes 2 d_k and, without
+the delta rule, b_i takes 2 d_v (both are bf16 inputs, stored exactly).  Token I/O: q and k (shared by the n_heads/n_kheads
 value heads of a group, so counted once per group), v, lambda (per step; a per-head
 constant costs nothing per step), beta (delta rule) and the fp32 output.
 """
@@ -21,8 +22,10 @@ from __future__ import annotations
 from .synth import Workload
 
 
-def entry_bytes(wl: Workload) -> int:
+def entry_bytes(wl: Workload, log_format: str = "fp32") -> int:
     lam = {"none": 0, "scalar": 4, "diag": 4 * wl.d_k}[wl.decay]
+    if log_format == "compact":
+        return 2 * wl.d_k + (4 if wl.update != "add" else 2) * wl.d_v + lam
     return 4 * wl.d_k + 4 * wl.d_v + lam
 
 
@@ -47,21 +50,21 @@ def eager_head_step(wl: Workload) -> float:
     return 2 * state_bytes(wl) + token_bytes(wl)
 
 
-def deferred_head_step(wl: Workload, c: int, merge: bool) -> float:
+def deferred_head_step(wl: Workload, c: int, merge: bool, log_format: str = "fp32") -> float:
     """One decode step of one head whose log holds c live entries."""
-    e = entry_bytes(wl)
+    e = entry_bytes(wl, log_format)
     if merge:
         return 2 * state_bytes(wl) + c * e + token_bytes(wl)
     return state_bytes(wl) + c * e + e + token_bytes(wl)
 
 
-def merge_head(wl: Workload, c: int) -> float:
-    return 2 * state_bytes(wl) + c * entry_bytes(wl)
+def merge_head(wl: Workload, c: int, log_format: str = "fp32") -> float:
+    return 2 * state_bytes(wl) + c * entry_bytes(wl, log_format)
 
 
-def deferred_cycle_average(wl: Workload) -> float:
+def deferred_cycle_average(wl: Workload, log_format: str = "fp32") -> float:
     """Per head-step bytes averaged over one merge interval (c = 0 .. L-1, the last
     step of the interval being the merge step)."""
     L = wl.log_cap
-    tot = sum(deferred_head_step(wl, c, merge=(c == L - 1)) for c in range(L))
+    tot = sum(deferred_head_step(wl, c, merge=(c == L - 1), log_format=log_format) for c in range(L))
     return tot / L

@@ -111,3 +111,39 @@ def gpu_rollout(runner: DecodeRunner, T: int, ckpts=(), layers=None, keep_inputs
     torch.cuda.synchronize()
     return ({l: np.stack(v) for l, v in outs.items()},
             {l: (np.stack(v) if v else None) for l, v in states.items()}, kept)
+
+
+def log_entries_f64(pool) -> np.ndarray:
+    """The pool's log ring as float64 [slot, layer, head, L, 2 d_k + d_v] rows
+    [a | b | Lambda], whatever its layout (test-side decoding of the compact layout:
+    bf16 a, bf16 b without the delta rule, Lambda fp32 x d_k / x 4 / none)."""
+    raw = pool.log.detach().cpu().contiguous()
+    dk, dv = pool.d_k, pool.d_v
+    if pool.log_format == "fp32":
+        return raw.double().numpy()
+    words = raw.view(torch.int32).numpy()
+    lead = words.shape[:-1]
+    out = np.zeros(lead + (2 * dk + dv,), np.float64)
+
+    def bf16(w):   # packed pairs of bf16 in 32-bit words -> float64
+        h = w.view(np.uint32)
+        lo = (h & np.uint32(0xFFFF)).astype(np.uint32) << np.uint32(16)
+        hi = h & np.uint32(0xFFFF0000)
+        return np.stack([lo.view(np.float32), hi.view(np.float32)], axis=-1).reshape(w.shape[:-1] + (-1,)).astype(np.float64)
+
+    def f32(w):
+        return w.view(np.float32).astype(np.float64)
+
+    out[..., :dk] = bf16(words[..., :dk // 2])
+    boff = dk // 2
+    if pool.update == "add":
+        out[..., dk:dk + dv] = bf16(words[..., boff:boff + dv // 2])
+        loff = boff + dv // 2
+    else:
+        out[..., dk:dk + dv] = f32(words[..., boff:boff + dv])
+        loff = boff + dv
+    if pool.decay == "diag":
+        out[..., dk + dv:] = f32(words[..., loff:loff + dk])
+    elif pool.decay == "scalar":
+        out[..., dk + dv] = f32(words[..., loff])
+    return out

@@ -9,8 +9,8 @@ import pytest
 from recurrent_state_serving_b200 import deltalog as dl
 
 EXPECTED = ["dl_append", "dl_create_pool", "dl_decode_step", "dl_decode_step_noalloc",
-            "dl_destroy_pool", "dl_eager_step", "dl_materialize", "dl_merge", "dl_read_error",
-            "dl_reset_slots", "dl_status_string"]
+            "dl_destroy_pool", "dl_eager_step", "dl_log_bytes", "dl_materialize", "dl_merge",
+            "dl_read_error", "dl_reset_slots", "dl_status_string"]
 
 
 def test_header_declares_the_boundary():
@@ -33,7 +33,7 @@ def test_only_the_abi_is_exported():
 
 def _desc(**kw):
     base = dict(n_slots=4, n_layers=2, n_heads=4, n_kheads=2, d_k=128, d_v=128, log_cap=8,
-                decay=2, update=1, tile_v=0, state=0x10000, log=0x20000, log_len=0x30000,
+                decay=2, update=1, tile_v=0, log_format=0, state=0x10000, log=0x20000, log_len=0x30000,
                 arrive=0x40000, err_word=0x50000)
     base.update(kw)
     return dl.dl_pool_desc(**base)
@@ -49,7 +49,8 @@ def test_create_pool_accepts_valid_descriptors():
     for kw in ({}, dict(d_k=16, d_v=16, n_kheads=4), dict(d_k=64, d_v=80), dict(log_cap=1),
                dict(log_cap=64), dict(log=None, log_len=None, arrive=None), dict(decay=0, update=0),
                dict(tile_v=16), dict(tile_v=32), dict(d_k=64, d_v=96, tile_v=32),
-               dict(tile_v=128, log_cap=32), dict(tile_v=128, log_cap=64)):
+               dict(tile_v=128, log_cap=32), dict(tile_v=128, log_cap=64), dict(log_format=1),
+               dict(log_format=1, decay=1, update=0, tile_v=128)):
         st, h = _create(_desc(**kw))
         assert st == dl.DL_OK, (kw, dl.dl_status_string(st))
         assert dl.library().dl_destroy_pool(h) == dl.DL_OK
@@ -78,6 +79,8 @@ def test_create_pool_accepts_valid_descriptors():
     (dict(tile_v=128, d_k=64, d_v=128), dl.DL_ERR_SHAPE),
     (dict(tile_v=128, d_v=256), dl.DL_ERR_SHAPE),
     (dict(tile_v=64), dl.DL_ERR_SHAPE),
+    (dict(log_format=2), dl.DL_ERR_INVALID_ARG),
+    (dict(log_format=-1), dl.DL_ERR_INVALID_ARG),
 ])
 def test_create_pool_rejects(kw, status):
     st, h = _create(_desc(**kw))
@@ -167,3 +170,43 @@ def test_noalloc_entry_point_checks_without_gpu():
     assert call(arrive=None, n_slots=65536, n_layers=2) == dl.DL_ERR_SHAPE   # > 65536 counters
     assert call(arrive=None, n_slots=32768, n_layers=2) == dl.DL_OK
     assert lib.dl_decode_step_noalloc(None, 0, ctypes.byref(a), 1, None) == dl.DL_ERR_INVALID_ARG
+
+
+def test_log_bytes_per_layout():
+    """dl_log_bytes: rows x entry bytes of the layout (fp32 [a|b|Lambda], or compact with
+    bf16 a, bf16 b without the delta rule, and Lambda per key / 4 floats / none)."""
+    lib = dl.library()
+    rows = 4 * 2 * 4 * 8
+
+    def nbytes(**kw):
+        n = ctypes.c_int64(-1)
+        d = _desc(**kw)
+        return lib.dl_log_bytes(ctypes.byref(d), ctypes.byref(n)), n.value
+
+    for decay in (0, 1, 2):
+        for update in (0, 1, 2):
+            assert nbytes(decay=decay, update=update) == (dl.DL_OK, rows * 4 * (2 * 128 + 128))
+    entry = {(0, 0): 512, (0, 1): 768, (1, 0): 528, (1, 1): 784, (2, 0): 1024, (2, 1): 1280}
+    for (decay, update), e in entry.items():
+        assert nbytes(decay=decay, update=update, log_format=1) == (dl.DL_OK, rows * e)
+        assert e % 16 == 0
+    assert nbytes(decay=2, update=2, log_format=1) == (dl.DL_OK, rows * 1280)
+    assert nbytes(d_k=16, d_v=48, decay=1, update=0, log_format=1) == (dl.DL_OK, rows * (32 + 96 + 16))
+    assert nbytes(log_format=3)[0] == dl.DL_ERR_INVALID_ARG
+    assert nbytes(d_v=40)[0] == dl.DL_ERR_SHAPE
+    assert lib.dl_log_bytes(None, None) == dl.DL_ERR_INVALID_ARG
+
+
+def test_compact_log_needs_bf16_inputs():
+    """A compact log stores k_t (and v_t) in bf16, exact only for bf16 inputs: decode and
+    append steps with fp32 q/k/v are refused on the host."""
+    lib = dl.library()
+    st, h = _create(_desc(log_format=1))
+    assert st == dl.DL_OK
+    P = 0x60000
+    a = dl.dl_step_args(P, 2, P, P, P, 0, P, 0, P, P)   # in_dtype = fp32
+    assert lib.dl_decode_step(h, 0, ctypes.byref(a), 1, None) == dl.DL_ERR_DTYPE
+    assert lib.dl_append(h, 0, ctypes.byref(a), None) == dl.DL_ERR_DTYPE
+    d = _desc(log_format=1, arrive=None)
+    assert lib.dl_decode_step_noalloc(ctypes.byref(d), 0, ctypes.byref(a), 1, None) == dl.DL_ERR_DTYPE
+    lib.dl_destroy_pool(h)

@@ -25,10 +25,10 @@ REDUCED = {
     "retnet": synth.RETNET.with_(n_layers=2, batch=7, n_heads=4, n_kheads=4, steps=256),
     # 128 x 128 heads without decay (linear attention, DeltaNet)
     "la_d128": synth.TINY_LA.with_(batch=3, n_heads=3, n_kheads=3, d_k=128, d_v=128, steps=96,
-                                   log_cap=12, qkv_std=1 / np.sqrt(128), init_std=0.02),
+                                   log_cap=12, qkv_std=1 / np.sqrt(128), init_std=0.02, in_dtype="bf16"),
     "deltanet_d128": synth.TINY_LA.with_(batch=3, n_heads=3, n_kheads=3, d_k=128, d_v=128, steps=96,
                                          log_cap=12, qkv_std=1 / np.sqrt(128), init_std=0.02,
-                                         update="delta", k_l2norm=True),
+                                         update="delta", k_l2norm=True, in_dtype="bf16"),
     # long logs: a merge of exactly 32 entries, and merges of more than 32 entries
     "kda_L33": synth.KDA.with_(n_layers=1, batch=3, n_heads=3, n_kheads=3, steps=140, log_cap=33),
     "gla_L64": synth.GLA_DIAG.with_(batch=2, n_heads=3, n_kheads=3, steps=200, log_cap=64,
@@ -39,11 +39,11 @@ REDUCED = {
 }
 
 
-def _run_case(wl, update=None, slot_seed=0, extra_slots=3, tile_v=0):
+def _run_case(wl, update=None, slot_seed=0, extra_slots=3, tile_v=0, log_format="fp32"):
     T = wl.steps
     ck = sorted({0, 1, T // 2, T})
     r = DecodeRunner(wl, n_slots=wl.batch + extra_slots, slot_seed=slot_seed, update=update,
-                     tile_v=tile_v)
+                     tile_v=tile_v, log_format=log_format)
     outs, states, _ = H.gpu_rollout(r, T, ckpts=ck)
     assert r.errors() == 0
     for layer in r.layers:
@@ -121,15 +121,16 @@ def test_log_cap_one_is_eager_bit_for_bit(tile_v):
     assert int(rd.pool.log_len.abs().sum()) == 0
 
 
+@pytest.mark.parametrize("log_format", ["fp32", "compact"])
 @pytest.mark.parametrize("tile_v", [16, 128])
-def test_log_contents_match_the_deferred_oracle(tile_v):
+def test_log_contents_match_the_deferred_oracle(tile_v, log_format):
     """Entry i of the ring holds (a_i, b_i, Lambda_i) exactly as the paper's log does."""
     from oracle.deferred import DeferredHead
     wl = synth.KDA.with_(n_layers=1, batch=2, n_heads=2, n_kheads=2, steps=11, log_cap=8)
-    r = DecodeRunner(wl, tile_v=tile_v)
+    r = DecodeRunner(wl, tile_v=tile_v, log_format=log_format)
     _, _, inputs = H.gpu_rollout(r, wl.steps, keep_inputs=True)
     S0 = synth.initial_state(wl, 0)
-    log = r.pool.log.double().cpu().numpy()
+    log = H.log_entries_f64(r.pool)
     live = r.pool.log_len.cpu().numpy()
     f = lambda x: synth.input_to_f64(x, wl.in_dtype)
     dk, dv = wl.d_k, wl.d_v
@@ -309,3 +310,73 @@ def test_fullsize_retnet_b1024_sampled_rows():
     H.check_steps(outs[3][:, rows], O)
     del r
     torch.cuda.empty_cache()
+
+
+# ---- compact log layout (bf16 a_i, bf16 b_i without the delta rule) ----------------
+COMPACT_CASES = [n for n in sorted(REDUCED) if REDUCED[n].in_dtype == "bf16"]
+
+
+@pytest.mark.parametrize("tile_v", [16, 32, 128])
+@pytest.mark.parametrize("name", COMPACT_CASES)
+def test_compact_log_parity_vs_oracle(name, tile_v):
+    wl = REDUCED[name]
+    if not _tile_ok(wl, tile_v) or (tile_v == 32 and name not in ("gla_L8", "kda", "retnet", "gdn_gva")):
+        pytest.skip("tile width not applicable (or covered by the other widths)")
+    _run_case(wl, tile_v=tile_v, log_format="compact")
+
+
+@pytest.mark.parametrize("tile_v", [16, 32, 128])
+@pytest.mark.parametrize("name", ["gla_L8", "kda", "retnet", "gdn_gva_256", "deltanet_d128"])
+def test_compact_log_matches_fp32_log(name, tile_v):
+    """The compact layout stores the same values (bf16 inputs, exactly), so a compact
+    pool computes what an fp32 pool does: bit for bit on the value-tiled kernels, whose
+    order of summation is the same; within the GPU deferred tolerance on the whole-head
+    kernel, whose stages hold a different number of entries per layout."""
+    wl = REDUCED[name]
+    if not _tile_ok(wl, tile_v):
+        pytest.skip("tile width not applicable")
+    T = min(wl.steps, 96)
+    res = {}
+    for fmt in ("fp32", "compact"):
+        r = DecodeRunner(wl, n_slots=wl.batch + 1, slot_seed=2, tile_v=tile_v, log_format=fmt)
+        res[fmt] = H.gpu_rollout(r, T, ckpts=[T])
+        assert r.errors() == 0
+    for layer in res["fp32"][0]:
+        of, sf = res["fp32"][0][layer], res["fp32"][1][layer]
+        oc, sc = res["compact"][0][layer], res["compact"][1][layer]
+        if tile_v in (16, 32):
+            np.testing.assert_array_equal(oc, of)
+            np.testing.assert_array_equal(sc, sf)
+        else:
+            H.check_steps(oc, of, tol=H.REL_L2_GPU, elem=None, what="compact vs fp32 output")
+            H.check_steps(sc, sf, tol=H.REL_L2_GPU, elem=None, what="compact vs fp32 state")
+
+
+def test_compact_log_append_merge_and_materialize():
+    """dl_append / dl_merge / dl_materialize read and write the compact layout."""
+    wl = synth.GLA_DIAG.with_(batch=3, n_heads=3, n_kheads=3, steps=20, log_cap=6)
+    out = {}
+    for fmt in ("fp32", "compact"):
+        r = DecodeRunner(wl, n_slots=4, slot_seed=5, log_format=fmt, tile_v=16)
+        r.load_initial_state()
+        seen = []
+        for t in range(wl.steps):
+            x = r.gen_inputs(t, 0)
+            if t % 6 < 5:
+                dl.dl_append(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"])
+            else:
+                dl.dl_merge(r.pool, 0, r.slots)
+            seen.append(r.materialize(0).double().cpu().numpy())
+        assert r.errors() == 0
+        out[fmt] = np.stack(seen)
+    np.testing.assert_array_equal(out["compact"], out["fp32"])
+
+
+def test_compact_log_refuses_fp32_inputs_on_gpu():
+    wl = synth.TINY_LA.with_(d_k=128, d_v=128, n_heads=2, n_kheads=2, batch=2)
+    r = DecodeRunner(wl, log_format="compact")
+    r.load_initial_state()
+    x = r.gen_inputs(0, 0)   # fp32 q/k/v
+    with pytest.raises(dl.DeltaLogError) as e:
+        r.call(0, x)
+    assert e.value.status == dl.DL_ERR_DTYPE
