@@ -101,6 +101,16 @@ __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// ---- Programmatic dependent launch.  griddep_wait blocks until the grid this one
+// depends on (the previous kernel in the stream, when launched with programmatic
+// stream serialization) has completed and its memory is visible; without such a
+// dependency it returns at once.  griddep_launch_dependents lets the next grid begin
+// launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- Tensor memory (TMEM): 128 lanes x 512 columns of 32-bit cells per SM.
 // Allocation is per CTA, in columns (a power of two >= 32), by one whole warp; the
 // address of the first column is written to shared memory.  A warp reaches only

@@ -206,6 +206,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     ptx::tmem_fence_before_sync();
     __syncthreads();
     ptx::tmem_fence_after_sync();
+    // Only on-chip state was touched so far.  With programmatic dependent launch this
+    // CTA may have started while the previous kernel in the stream was finishing:
+    // global memory is read only after that kernel has completed.  The next launch
+    // may then begin (its CTAs take an SM only when this one leaves it).
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     // this warp's TMEM: lanes of its quarter, columns of its half
     const uint32_t tm = use_tm ? *tm_slot + ((uint32_t)(32 * (w & 3)) << 16) + TM_WCOLS * (uint32_t)(w >> 2)
                                : 0u;

@@ -38,7 +38,21 @@ cudaError_t launch_one(const KParams &p, cudaStream_t st) {
     const long long items = (long long)p.batch * p.H;
     const long long sms = device_sm_count();
     const int grid = (int)(items < sms ? items : sms);
-    kern<<<grid, wh::NTHREADS, wh::SMEM, st>>>(p);
+    // programmatic stream serialization: the launch may overlap the end of the
+    // previous kernel in the stream; the kernel waits for it (griddepcontrol.wait)
+    // before its first global memory access
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(wh::NTHREADS);
+    cfg.dynamicSmemBytes = wh::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
