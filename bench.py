@@ -82,6 +82,8 @@ def parse():
                     help="cold L2 per step: rotate slot groups (inputs > L2) or flush before each step")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="rotate mode: replay the timed steps from a CUDA graph or launch them directly")
+    ap.add_argument("--replay", default="per_tile", choices=["per_tile", "cluster"],
+                    help="value-tiled kernel: ReplayPrep formed per tile, or shared by a head's tiles as one cluster")
     ap.add_argument("--log-format", default="fp32", choices=["fp32", "compact"],
                     help="log entry layout: fp32 [a|b|Lambda], or compact (bf16 a, bf16 b without the delta rule)")
     return ap.parse_args()
@@ -117,10 +119,10 @@ def l2_description(wl, l2_mode: str, launch: str) -> str:
             f"{'replayed from one CUDA graph' if launch == 'graph' else 'launched directly'}")
 
 
-def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph", log_format="fp32"):
+def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph", log_format="fp32", replay="per_tile"):
     suffix = "" if log_format == "fp32" else f"_{log_format}log"
     return {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}{suffix}",
-            "tile_v": tile_v or "auto", "log_format": log_format,
+            "tile_v": tile_v or "auto", "log_format": log_format, "replay": replay,
             "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
             "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
             "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
@@ -393,7 +395,8 @@ def run_gpu(a, wl, rank, world, dist):
         return ms
 
     # ---- deferred (the product path) ----
-    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format)
+    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format,
+                     replay=a.replay)
     r.load_initial_state()
     r.run_presteps()
     dev_inputs = [[r.device_inputs(x) for x in per_layer] for per_layer in host_inputs]
@@ -579,7 +582,7 @@ def run_reference(a, wl):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch, a.log_format),
+            "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch, a.log_format, a.replay),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -626,7 +629,7 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; bf16 q/k/v, fp32 lambda/beta, fp32 state and log)",
-            "config": config_of(wl, world, a.tile_v, a.l2, a.launch, a.log_format), "roofline": res["roofline"],
+            "config": config_of(wl, world, a.tile_v, a.l2, a.launch, a.log_format, a.replay), "roofline": res["roofline"],
             "gpu_launches": res["gpu_launches"],
             "hbm_tbs": res["roofline"]["achieved"] / 1e3}
     for k in ("eager", "deferred_bytes_per_step", "e2e", "clocks", "rotation_groups", "graph_uploaded"):

@@ -93,6 +93,20 @@ typedef enum { DL_F32 = 0, DL_BF16 = 1 } dl_dtype;
  * dl_log_bytes gives the size of the log buffer either layout needs. */
 typedef enum { DL_LOG_FP32 = 0, DL_LOG_COMPACT = 1 } dl_log_format;
 
+/* Where the value-tiled kernel forms the key-side replay coefficients (ReplayPrep,
+ * Section 3.3: q^T A'_i and k^T A'_i, with A'_i for a merge).  The whole-head kernel
+ * (tile_v 128) always forms them once per head, in the head's warp.
+ *  DL_REPLAY_PER_TILE  every value tile forms all of them itself (default; the fused,
+ *                      redundant form).
+ *  DL_REPLAY_CLUSTER   the d_v / B_V tiles of a head run as one thread-block cluster
+ *                      (when that is 2..8 CTAs); each tile forms a share of the entries
+ *                      and reads the rest from the others' shared memory.
+ * Measured on B200 the cluster form is slower for most launches (co-scheduling the
+ * cluster and its two barriers cost more than the redundant replay) and faster only
+ * for the smallest launches with long logs; it is kept for that case and for the
+ * ablation of Section 3.3's staged ReplayPrep. */
+typedef enum { DL_REPLAY_PER_TILE = 0, DL_REPLAY_CLUSTER = 1 } dl_replay_mode;
+
 /* Sticky device error bits (dl_read_error). */
 #define DL_EBIT_SLOT_RANGE 0x1  /* a slot id outside [0, n_slots)                    */
 #define DL_EBIT_LOG_FULL 0x2    /* append / decode without auto-merge on a full log   */
@@ -132,6 +146,7 @@ typedef enum { DL_LOG_FP32 = 0, DL_LOG_COMPACT = 1 } dl_log_format;
  *           unless that leaves SMs idle, else 16).  32 needs d_k >= 64 and d_v a
  *           multiple of 32.
  *  log_format dl_log_format of the log (DL_LOG_FP32 or DL_LOG_COMPACT).
+ *  replay_mode dl_replay_mode (DL_REPLAY_PER_TILE or DL_REPLAY_CLUSTER).
  *
  * The cumulative log-decay lbar of a slot is not stored separately: it equals
  * Lambda of the newest live entry (0 when the log is empty).
@@ -141,7 +156,8 @@ typedef struct {
     dl_decay decay;
     dl_update update;
     int32_t tile_v;
-    int32_t log_format;  /* dl_log_format */
+    int32_t log_format;   /* dl_log_format */
+    int32_t replay_mode;  /* dl_replay_mode */
     float *state;
     float *log;
     int32_t *log_len;

@@ -65,6 +65,7 @@ dl::KParams base_params(const dl_pool_desc &d, int layer) {
     p.a16 = l.a16;
     p.b16 = l.b16;
     p.layer = layer;
+    p.cl = 1;
     return p;
 }
 
@@ -138,6 +139,9 @@ dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_o
     } else {
         int bv = 32;
         set_tiles(d, p, a->batch, bv);
+        // ReplayPrep shared by the head's value tiles as one cluster (2..8 CTAs); an
+        // eager step has no log to replay
+        p.cl = (d.replay_mode == DL_REPLAY_CLUSTER && !eager && p.nv >= 2 && p.nv <= 8) ? p.nv : 1;
         e = dl::launch_step(p, bv, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
                             static_cast<cudaStream_t>(stream));
     }
@@ -177,6 +181,7 @@ DL_API dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool) {
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;
     if (d.log_format != DL_LOG_FP32 && d.log_format != DL_LOG_COMPACT) return DL_ERR_INVALID_ARG;
+    if (d.replay_mode != DL_REPLAY_PER_TILE && d.replay_mode != DL_REPLAY_CLUSTER) return DL_ERR_INVALID_ARG;
     if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
         return DL_ERR_INVALID_ARG;
     if (d.log && (!aligned(d.log, 16) || !d.log_len || !d.arrive)) return DL_ERR_INVALID_ARG;
@@ -313,6 +318,7 @@ dl_status check_desc_without_arrive(const dl_pool_desc &d) {
     if ((int)d.update < DL_UPDATE_ADD || (int)d.update > DL_UPDATE_DELTA_UNDECAYED)
         return DL_ERR_INVALID_ARG;
     if (d.log_format != DL_LOG_FP32 && d.log_format != DL_LOG_COMPACT) return DL_ERR_INVALID_ARG;
+    if (d.replay_mode != DL_REPLAY_PER_TILE && d.replay_mode != DL_REPLAY_CLUSTER) return DL_ERR_INVALID_ARG;
     if (!d.state || !aligned(d.state, 16) || !d.err_word || !aligned(d.err_word, 4))
         return DL_ERR_INVALID_ARG;
     if (!d.log || !aligned(d.log, 16) || !d.log_len || !aligned(d.log_len, 4))

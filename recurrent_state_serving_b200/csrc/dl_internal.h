@@ -24,6 +24,7 @@ struct KParams {
     int loff;   // offset of Lambda_i in an entry, in floats
     int a16;    // a_i stored as bf16 (compact layout)
     int b16;    // b_i stored as bf16 (compact layout without the delta rule)
+    int cl;     // value tiles of a head sharing ReplayPrep as one cluster (1: each alone)
     int nv;     // value tiles per head: d_v / B_V
     int layer;
     // batch

@@ -14,6 +14,7 @@
 // while the CTA computes its replay coefficients.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -129,9 +130,18 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     const int bi = blockIdx.x / (nv * p.H);
     const int dv = p.dv;
 
+    // A CTA that leaves early still passes the two cluster barriers its tiles wait
+    // at below, so a call whose tiles disagree (slots not distinct) cannot hang them.
+    auto leave = [&]() {
+        if (p.cl > 1) {
+            cooperative_groups::this_cluster().sync();
+            cooperative_groups::this_cluster().sync();
+        }
+    };
     const int s = p.slots[bi];
     if (s < 0 || s >= p.n_slots) {
         if (tid == 0) atomicOr(p.err, DL_EBIT_SLOT_RANGE);
+        leave();
         return;
     }
     const size_t sl = (size_t)s * p.n_layers + p.layer;
@@ -154,15 +164,18 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     if (p.eager) {
         if (c != 0) {
             if (tid == 0) atomicOr(p.err, DL_EBIT_LIVE_LOG);
+            leave();
             return;
         }
     } else if (c < 0 || c > p.L) {
         if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_LEN);
+        leave();
         return;
     }
     const bool merge_now = p.eager || (p.auto_merge && c >= p.L - 1);
     if (!merge_now && c >= p.L) {
         if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_FULL);
+        leave();
         return;
     }
     float *ring = p.log ? p.log + head * (size_t)p.L * p.E : nullptr;
@@ -203,8 +216,12 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     }
     __syncthreads();
 
-    // 4. ReplayPrep: key-side replay coefficients, one warp per log entry
-    for (int i = warp; i < c; i += NW) {
+    // 4. ReplayPrep: key-side replay coefficients, one warp per log entry.  With
+    //    p.cl > 1 the head's p.cl value tiles run as one thread-block cluster and
+    //    tile j forms the entries of warps j*NW .. j*NW + NW-1 of each round; the
+    //    tiles read the rest from one another below.
+    const int cl = p.cl, cr = p.cl > 1 ? j : 0;
+    for (int i = cr * NW + warp; i < c; i += NW * cl) {
         const float *ent = ring + (size_t)i * p.E;
         float fs = 1.f, fk = 1.f;
         if (DECAY == DL_DECAY_SCALAR) {
@@ -254,6 +271,27 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         if (lane == 0) s_kq = x;
     }
     __syncthreads();
+    if (cl > 1) {
+        // coefficients (and, on a merge step, A' rows) formed by the other tiles
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        for (int i = tid; i < c; i += NT) {
+            const int o = (i / NW) % cl;
+            if (o != cr) {
+                s_cq[i] = *cluster.map_shared_rank(s_cq + i, o);
+                if (DELTA) s_ck[i] = *cluster.map_shared_rank(s_ck + i, o);
+            }
+        }
+        if (merge_now) {
+            for (int idx = tid; idx < c * DK; idx += NT) {
+                const int o = (idx / DK / NW) % cl;
+                if (o != cr) s_A[idx] = *cluster.map_shared_rank(s_A + idx, o);
+            }
+        }
+        // no tile moves on (or leaves) while another still reads its shared memory
+        cluster.sync();
+    }
 
     // 5. AppendDecode: base mat-vecs S^T qt and S^T kt over this tile
     float yq[4] = {0.f, 0.f, 0.f, 0.f}, yk[4] = {0.f, 0.f, 0.f, 0.f};

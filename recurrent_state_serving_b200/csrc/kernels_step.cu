@@ -16,7 +16,26 @@ cudaError_t launch_one(const KParams &p, cudaStream_t st) {
     using Sh = TileShape<DL_STEP_DK, BV>;
     const size_t smem = dyn_floats(p.L, DL_STEP_DK, BV, p.auto_merge != 0) * sizeof(float);
     const long long grid = (long long)p.batch * p.H * p.nv;
-    step_kernel<DL_STEP_DK, BV, DECAY, DELTA, IT><<<(unsigned)grid, Sh::NT, smem, st>>>(p);
+    auto kern = step_kernel<DL_STEP_DK, BV, DECAY, DELTA, IT>;
+    if (p.cl <= 1) {
+        kern<<<(unsigned)grid, Sh::NT, smem, st>>>(p);
+        return cudaGetLastError();
+    }
+    // a head's p.cl = p.nv value tiles (adjacent in blockIdx) as one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(Sh::NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -30,6 +30,7 @@ DECAY = {"none": 0, "scalar": 1, "diag": 2}
 UPDATE = {"add": 0, "delta": 1, "delta_undecayed": 2}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 LOG_FORMAT = {"fp32": 0, "compact": 1}
+REPLAY = {"per_tile": 0, "cluster": 1}
 DL_EBIT_SLOT_RANGE, DL_EBIT_LOG_FULL, DL_EBIT_LIVE_LOG, DL_EBIT_LOG_LEN, DL_EBIT_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
 
@@ -39,7 +40,8 @@ class dl_pool_desc(ctypes.Structure):
                 ("n_heads", ctypes.c_int32), ("n_kheads", ctypes.c_int32),
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("log_cap", ctypes.c_int32),
                 ("decay", ctypes.c_int), ("update", ctypes.c_int), ("tile_v", ctypes.c_int32),
-                ("log_format", ctypes.c_int32), ("state", ctypes.c_void_p), ("log", ctypes.c_void_p),
+                ("log_format", ctypes.c_int32), ("replay_mode", ctypes.c_int32),
+                ("state", ctypes.c_void_p), ("log", ctypes.c_void_p),
                 ("log_len", ctypes.c_void_p), ("arrive", ctypes.c_void_p),
                 ("err_word", ctypes.c_void_p)]
 
@@ -123,14 +125,15 @@ class Pool:
 
     def __init__(self, n_slots, n_layers, n_heads, d_k, d_v, log_cap, decay="none",
                  update="add", n_kheads=None, device="cuda", with_log=True, tile_v=0,
-                 log_format="fp32"):
+                 log_format="fp32", replay="per_tile"):
         dev = torch.device(device)
         n_kheads = n_heads if n_kheads is None else n_kheads
         self.n_slots, self.n_layers, self.n_heads, self.n_kheads = n_slots, n_layers, n_heads, n_kheads
         self.d_k, self.d_v, self.log_cap, self.decay, self.update = d_k, d_v, log_cap, decay, update
-        self.tile_v, self.log_format = tile_v, log_format
+        self.tile_v, self.log_format, self.replay = tile_v, log_format, replay
         self.desc = dl_pool_desc(n_slots, n_layers, n_heads, n_kheads, d_k, d_v, log_cap,
-                                 DECAY[decay], UPDATE[update], tile_v, LOG_FORMAT[log_format])
+                                 DECAY[decay], UPDATE[update], tile_v, LOG_FORMAT[log_format],
+                                 REPLAY[replay])
         nbytes = ctypes.c_int64()
         _check(_lib.dl_log_bytes(ctypes.byref(self.desc), ctypes.byref(nbytes)), "dl_log_bytes")
         # one entry in 4-byte words (its bf16 parts, if any, are packed in pairs)

@@ -35,7 +35,8 @@ def _to_dev_input(a, in_dtype, device):
 class DecodeRunner:
     def __init__(self, wl: synth.Workload, *, n_slots: int | None = None, slot_seed: int | None = None,
                  layers=None, mode: str = "deferred", update: str | None = None,
-                 device: str = "cuda", tile_v: int = 0, n_groups: int = 1, log_format: str = "fp32"):
+                 device: str = "cuda", tile_v: int = 0, n_groups: int = 1, log_format: str = "fp32",
+                 replay: str = "per_tile"):
         if mode not in ("deferred", "eager"):
             raise ValueError(mode)
         self.wl = wl
@@ -57,7 +58,7 @@ class DecodeRunner:
         self.pool = dl.Pool(n_slots * n_groups, wl.n_layers, wl.n_heads, wl.d_k, wl.d_v, wl.log_cap,
                             decay=wl.decay, update=self.update, n_kheads=wl.n_kheads,
                             device=device, with_log=(mode == "deferred"), tile_v=tile_v,
-                            log_format=log_format)
+                            log_format=log_format, replay=replay)
         self.offsets = synth.slot_offsets(wl)
 
     # -- set-up ----------------------------------------------------------------

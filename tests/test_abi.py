@@ -33,7 +33,7 @@ def test_only_the_abi_is_exported():
 
 def _desc(**kw):
     base = dict(n_slots=4, n_layers=2, n_heads=4, n_kheads=2, d_k=128, d_v=128, log_cap=8,
-                decay=2, update=1, tile_v=0, log_format=0, state=0x10000, log=0x20000, log_len=0x30000,
+                decay=2, update=1, tile_v=0, log_format=0, replay_mode=0, state=0x10000, log=0x20000, log_len=0x30000,
                 arrive=0x40000, err_word=0x50000)
     base.update(kw)
     return dl.dl_pool_desc(**base)
@@ -50,7 +50,7 @@ def test_create_pool_accepts_valid_descriptors():
                dict(log_cap=64), dict(log=None, log_len=None, arrive=None), dict(decay=0, update=0),
                dict(tile_v=16), dict(tile_v=32), dict(d_k=64, d_v=96, tile_v=32),
                dict(tile_v=128, log_cap=32), dict(tile_v=128, log_cap=64), dict(log_format=1),
-               dict(log_format=1, decay=1, update=0, tile_v=128)):
+               dict(log_format=1, decay=1, update=0, tile_v=128), dict(replay_mode=1)):
         st, h = _create(_desc(**kw))
         assert st == dl.DL_OK, (kw, dl.dl_status_string(st))
         assert dl.library().dl_destroy_pool(h) == dl.DL_OK
@@ -81,6 +81,7 @@ def test_create_pool_accepts_valid_descriptors():
     (dict(tile_v=64), dl.DL_ERR_SHAPE),
     (dict(log_format=2), dl.DL_ERR_INVALID_ARG),
     (dict(log_format=-1), dl.DL_ERR_INVALID_ARG),
+    (dict(replay_mode=2), dl.DL_ERR_INVALID_ARG),
 ])
 def test_create_pool_rejects(kw, status):
     st, h = _create(_desc(**kw))

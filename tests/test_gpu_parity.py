@@ -380,3 +380,24 @@ def test_compact_log_refuses_fp32_inputs_on_gpu():
     with pytest.raises(dl.DeltaLogError) as e:
         r.call(0, x)
     assert e.value.status == dl.DL_ERR_DTYPE
+
+
+# ---- ReplayPrep shared by a head's value tiles (cluster) vs formed by every tile ----
+@pytest.mark.parametrize("tile_v", [16, 32])
+@pytest.mark.parametrize("name", ["gla_L8", "kda", "retnet", "gdn_gva_256", "deltanet_d128", "kda_L33"])
+def test_cluster_replay_matches_per_tile_bit_for_bit(name, tile_v):
+    """The tiles of a cluster form the same coefficients the per-tile form does, with
+    the same arithmetic, and read them from one another unchanged: results agree bit
+    for bit (decode steps with merges; both log layouts' value-tiled kernels)."""
+    wl = REDUCED[name]
+    if not _tile_ok(wl, tile_v):
+        pytest.skip("tile width not applicable")
+    T = min(wl.steps, 80)
+    res = {}
+    for mode in ("cluster", "per_tile"):
+        r = DecodeRunner(wl, n_slots=wl.batch + 1, slot_seed=4, tile_v=tile_v, replay=mode)
+        res[mode] = H.gpu_rollout(r, T, ckpts=[T])
+        assert r.errors() == 0
+    for layer in res["cluster"][0]:
+        np.testing.assert_array_equal(res["cluster"][0][layer], res["per_tile"][0][layer])
+        np.testing.assert_array_equal(res["cluster"][1][layer], res["per_tile"][1][layer])
