@@ -507,14 +507,14 @@ def run_gpu(a, wl, rank, world, dist):
 # ---------------------------------------------------------------------------------
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------------
-def oracle_sample_rate(wl, target_s=10.0):
+def oracle_sample_rate(wl, target_s=10.0, threads=None):
     """fp64 eager oracle on the host cores over a bounded sample of the workload's
     heads (layer 0); returns (head-steps/s, threads, description).  Up to 64
     distinct seeded steps are generated and cycled to reach about target_s of
-    oracle work; only the oracle call is timed."""
+    oracle work; only the oracle call is timed.  threads: all host cores by default."""
     import oracle
     from recurrent_state_serving_b200 import synth
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     S0 = synth.initial_state(wl.with_(batch=min(wl.batch, 64)), 0).astype(np.float64)
     rows = np.arange(S0.shape[0])
     ndist = min(64, wl.steps)
@@ -637,8 +637,9 @@ def main():
             line[k] = res[k]
     if world == 1 and not a.no_cpu:
         rate, cores, desc = oracle_sample_rate(wl)
+        rate1, _, desc1 = oracle_sample_rate(wl, target_s=3.0, threads=1)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": desc}
+                                "sample": desc, "value_1core": rate1, "sample_1core": desc1}
     print(json.dumps(line), flush=True)
 
 
