@@ -11,11 +11,11 @@
 // Lane l owns rows 4l..4l+3 for the key-side vectors (q, k, lbar_t, a_i,
 // Lambda_i, A'_i) and columns 4l..4l+3 for the value side (v, b_i, o_t, and the
 // mat-vec accumulators).  The mat-vecs S^T qt and S^T kt need every row's qt/kt
-// in every lane: they come from the owning lane by warp shuffle, so each lane
-// accumulates its four columns over all 128 rows with no cross-lane reduction.
-// Replay dot products (q^T A'_i, k^T A'_i) are warp butterfly sums.  Values a
-// row block needs in every lane (qt, kt, e^{lbar_t}, k and A'_i of its 16 rows) are
-// read as shared-memory broadcasts from a small per-warp area the owning lanes fill.
+// in every lane: the owning lanes write the head's row vectors (qt, kt, e^{lbar_t},
+// k, lbar_t) to a small per-warp shared-memory area once, and every lane reads
+// them as broadcasts, so each lane accumulates its four columns over all 128 rows
+// with no cross-lane reduction.  Replay dot products (q^T A'_i, k^T A'_i) are warp
+// butterfly sums.
 //
 // One stream per warp.  Each warp has a ring of NSW shared-memory stages of 8 KB;
 // lane 0 keeps NSW copies in flight with cp.async.bulk (TMA bulk copies, mbarrier
@@ -43,6 +43,12 @@
 // costs several append heads, and started early it overlaps their streaming instead
 // of ending the launch alone.  Warps then take heads in that order from a shared
 // counter.
+//
+// The kernel is instantiated per log layout (FMT 0: fp32 rows; FMT 1: compact rows,
+// bf16 a_i and, without the delta rule, bf16 b_i), which fixes how many entries a
+// stage carries and where each part of an entry sits.  It is launched with
+// programmatic stream serialization: a CTA sets up its mbarriers and TMEM while the
+// previous kernel in the stream finishes, and reads global memory only after it.
 //
 // Every wait is bounded (100 ms); a warp whose wait runs out sets
 // DL_EBIT_TIMEOUT, stops, and waits (bounded again) for its own copies still in
