@@ -221,42 +221,61 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     //    tile j forms the entries of warps j*NW .. j*NW + NW-1 of each round; the
     //    tiles read the rest from one another below.
     const int cl = p.cl, cr = p.cl > 1 ? j : 0;
-    for (int i = cr * NW + warp; i < c; i += NW * cl) {
-        const float *ent = ring + (size_t)i * p.E;
-        float fs = 1.f, fk = 1.f;
-        if (DECAY == DL_DECAY_SCALAR) {
-            const float Li = ent[p.loff];
-            fs = expf(s_ell[0] - Li);
-            fk = (DELTA && p.undecayed) ? expf(s_ellp[0] - Li) : fs;
-        }
-        float pq = 0.f, pk = 0.f;
-        for (int r4 = lane; r4 < DK / 4; r4 += 32) {
-            const float4 a4 = ent_a4(p, ent, r4);
-            float4 L4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (DECAY == DL_DECAY_DIAG) L4 = *reinterpret_cast<const float4 *>(ent + p.loff + 4 * r4);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-            const float Lv[4] = {L4.x, L4.y, L4.z, L4.w};
+    // A warp takes RU of its entries per round: their loads are all in flight before
+    // the first reduction, so a long log is not a chain of dependent round trips.
+    constexpr int RU = 4;
+    const int stride = NW * cl;
+    for (int i0 = cr * NW + warp; i0 < c; i0 += stride * RU) {
+        float pqv[RU], pkv[RU];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int r = 4 * r4 + x;
-                float w, wk;
-                if (DECAY == DL_DECAY_DIAG) {
-                    w = av[x] * expf(s_ell[r] - Lv[x]);
-                    wk = (DELTA && p.undecayed) ? av[x] * expf(s_ellp[r] - Lv[x]) : w;
-                } else {
-                    w = av[x] * fs;
-                    wk = av[x] * fk;
-                }
-                pq = fmaf(w, s_q[r], pq);
-                if (DELTA) pk = fmaf(wk, s_k[r], pk);
-                if (merge_now) s_A[i * DK + r] = w;
+        for (int u = 0; u < RU; ++u) {
+            pqv[u] = 0.f;
+            pkv[u] = 0.f;
+            const int i = i0 + u * stride;
+            if (i >= c) continue;
+            const float *ent = ring + (size_t)i * p.E;
+            float fs = 1.f, fk = 1.f;
+            if (DECAY == DL_DECAY_SCALAR) {
+                const float Li = ent[p.loff];
+                fs = expf(s_ell[0] - Li);
+                fk = (DELTA && p.undecayed) ? expf(s_ellp[0] - Li) : fs;
             }
+            float pq = 0.f, pk = 0.f;
+            for (int r4 = lane; r4 < DK / 4; r4 += 32) {
+                const float4 a4 = ent_a4(p, ent, r4);
+                float4 L4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (DECAY == DL_DECAY_DIAG) L4 = *reinterpret_cast<const float4 *>(ent + p.loff + 4 * r4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float Lv[4] = {L4.x, L4.y, L4.z, L4.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int r = 4 * r4 + x;
+                    float w, wk;
+                    if (DECAY == DL_DECAY_DIAG) {
+                        w = av[x] * expf(s_ell[r] - Lv[x]);
+                        wk = (DELTA && p.undecayed) ? av[x] * expf(s_ellp[r] - Lv[x]) : w;
+                    } else {
+                        w = av[x] * fs;
+                        wk = av[x] * fk;
+                    }
+                    pq = fmaf(w, s_q[r], pq);
+                    if (DELTA) pk = fmaf(wk, s_k[r], pk);
+                    if (merge_now) s_A[i * DK + r] = w;
+                }
+            }
+            pqv[u] = pq;
+            pkv[u] = pk;
         }
-        pq = warp_sum(pq);
-        if (DELTA) pk = warp_sum(pk);
-        if (lane == 0) {
-            s_cq[i] = pq;
-            s_ck[i] = pk;
+#pragma unroll
+        for (int u = 0; u < RU; ++u) {
+            const int i = i0 + u * stride;
+            if (i >= c) continue;
+            const float pq = warp_sum(pqv[u]);
+            const float pk = DELTA ? warp_sum(pkv[u]) : 0.f;
+            if (lane == 0) {
+                s_cq[i] = pq;
+                s_ck[i] = pk;
+            }
         }
     }
     // value-side log shard of this tile
