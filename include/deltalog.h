@@ -34,7 +34,12 @@
  * Streams.  Every call is asynchronous on the given cudaStream_t (passed as
  * void*, NULL = legacy default stream) except dl_read_error, which
  * synchronises that stream.  Calls on the same (pool, layer) must be ordered
- * on one stream; different layers may run concurrently.
+ * on one stream; different layers may run concurrently.  The whole-head decode
+ * kernel is launched with programmatic stream serialization: it may start while
+ * the previous kernel on its stream finishes, and reads no global memory before
+ * that kernel has completed.  Each of its CTAs (one per SM) holds all of that SM's
+ * tensor memory while it runs, so a kernel on another stream that holds tensor
+ * memory on the same SM delays it until those columns are released.
  *
  * Errors.  Argument problems found on the host are returned as a dl_status
  * before anything is launched.  Problems only the device can see (a slot id out
