@@ -41,8 +41,11 @@
 // of them than warps (and at most KMAX), the CTA first reads every head's slot id and
 // live length (all threads at once) and puts the merge steps first: a merge head
 // costs several append heads, and started early it overlaps their streaming instead
-// of ending the launch alone.  Warps then take heads in that order from a shared
-// counter.
+// of ending the launch alone.  A merge without the delta rule is split in two work
+// items, each streaming and rewriting half of the tile's rows (both stage the
+// coefficients in their own TMEM share); the second to finish adds the first's partial
+// output (left in `out`) to its own and commits the head.  Warps take the items in
+// that order from a shared counter.
 //
 // The kernel is instantiated per log layout (FMT 0: fp32 rows; FMT 1: compact rows,
 // bf16 a_i and, without the delta rule, bf16 b_i), which fixes how many entries a
@@ -80,10 +83,11 @@ constexpr int AG = 4;                       // merge entries per TMEM load / sha
 // per-warp scratch: the head's row vectors qt, kt, e^{lbar_t}, k, lbar_t (5 x 128 floats)
 // and the A' values of AG entries for the 16 rows of one block
 constexpr int WSCR = 5 * DK + AG * CR;
-// per-CTA head list: slot id, live length and the processing order of up to KMAX heads
+// per-CTA head list: slot id, live length, halves' combine state of up to KMAX heads,
+// and the processing order (a split merge head takes two positions)
 constexpr int KMAX = 512;
 constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4 + (size_t)NW * NB * 8 + 32 +
-                        (size_t)KMAX * (4 + 4 + 2);
+                        (size_t)KMAX * (4 + 4 + 4) + (size_t)2 * KMAX * 2;
 static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
 static_assert(TM_ENT * 8 <= (int)TM_WCOLS, "A'_i and b_i take 8 columns per entry");
 constexpr unsigned FULL = 0xffffffffu;
@@ -143,6 +147,7 @@ struct Head {
     int mk;        // MergeKind
     int nl;        // log chunks in its stream
     int n;         // stream positions: nl + NCH (+ NCH for MK_PASS2); 0 when skipped
+    int half;      // 0: the whole head; 1 / 2: rows 0..63 / 64..127 of a split merge
     size_t head;   // (slot, layer, head) index
 };
 
@@ -190,10 +195,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     uint64_t *pb = fb + NSW;  // round-wise merge: tile re-stream through stages 0 and 1
     int *next_k = reinterpret_cast<int *>(bars + (size_t)NW * NB * 8);
     uint32_t *tm_slot = reinterpret_cast<uint32_t *>(next_k + 1);
-    int *cnt = next_k + 2;  // merge heads, next merge position, next other position
+    int *cnt = next_k + 2;  // merge positions, next merge position, next other position, splits
     int *pre_slot = next_k + 8;
     int *pre_len = pre_slot + KMAX;
-    uint16_t *order = reinterpret_cast<uint16_t *>(pre_len + KMAX);
+    int *comb = pre_len + KMAX;  // split merge heads: halves arrived (1, 2) + 4 once a partial is in out
+    uint16_t *order = reinterpret_cast<uint16_t *>(comb + KMAX);  // k | half << 10
 
     // merges with live entries need tensor memory (auto-merge decode steps only)
     const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     }
     if (threadIdx.x == 0) {
         *next_k = NW;  // warp w starts with the CTA's w-th head
-        cnt[0] = cnt[1] = cnt[2] = 0;
+        cnt[0] = cnt[1] = cnt[2] = cnt[3] = 0;
     }
     if (use_tm && w == 0) {
         ptx::tmem_alloc(tm_slot, TM_COLS);
@@ -230,32 +236,55 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     auto merges = [&](int s, int c) {
         return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && c >= p.L - 1));
     };
+    // Merges written during pass 1 (no delta rule, at most TM_ENT entries) split in two
+    // when the CTA has few heads: a merge head costs about three append heads, so with
+    // fewer than three heads per warp it would outlast the rest of the CTA's work; with
+    // more, the other heads hide it and a split only adds the second half's log read.
+    const bool split_ok = kc < 3 * NW;
+    auto splits = [&](int s, int c) {
+        return split_ok && !DELTA && !p.eager && p.want_out && merges(s, c) && c >= 0 && c <= TM_ENT;
+    };
     if (pre) {
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
             const int s = p.slots[(bx + k * G) / p.H];
             const int c = (s >= 0 && s < p.n_slots && p.log_len) ? p.log_len[(size_t)s * p.n_layers + p.layer] : 0;
             pre_slot[k] = s;
             pre_len[k] = c;
-            if (merges(s, c)) atomicAdd(&cnt[0], 1);
+            comb[k] = 0;
+            if (merges(s, c)) atomicAdd(&cnt[0], splits(s, c) ? 2 : 1);
+            if (splits(s, c)) atomicAdd(&cnt[3], 1);
         }
         __syncthreads();
         const int nm = cnt[0];
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
-            const int pos = merges(pre_slot[k], pre_len[k]) ? atomicAdd(&cnt[1], 1) : nm + atomicAdd(&cnt[2], 1);
-            order[pos] = (uint16_t)k;
+            const int s = pre_slot[k], c = pre_len[k];
+            if (splits(s, c)) {
+                const int pos = atomicAdd(&cnt[1], 2);  // the two halves next to each other
+                order[pos] = (uint16_t)(k | (1 << 10));
+                order[pos + 1] = (uint16_t)(k | (2 << 10));
+            } else {
+                const int pos = merges(s, c) ? atomicAdd(&cnt[1], 1) : nm + atomicAdd(&cnt[2], 1);
+                order[pos] = (uint16_t)k;
+            }
         }
         __syncthreads();
     }
-    auto item_at = [&](int pos) -> int {
-        if (pos >= kc) return n_items;
-        return bx + (pre ? (int)order[pos] : pos) * G;
+    const int npos = pre ? kc + cnt[3] : kc;  // work items of this CTA
+    // work item at a position of the order: the head's item index and its half
+    auto item_at = [&](int pos, int &half) -> int {
+        half = 0;
+        if (pos >= npos) return n_items;
+        if (!pre) return bx + pos * G;
+        const int o = order[pos];
+        half = o >> 10;
+        return bx + (o & 1023) * G;
     };
     // warps take the next position from a shared counter as they finish, so a warp
     // held up by a merge head takes fewer heads
-    auto grab = [&]() -> int {
+    auto grab = [&](int &half) -> int {
         int pos = 0;
         if (lane == 0) pos = atomicAdd(next_k, 1);
-        return item_at(__shfl_sync(FULL, pos, 0));
+        return item_at(__shfl_sync(FULL, pos, 0), half);
     };
     const int E = p.E;
     const uint64_t pol_stream = ptx::policy_evict_first();
@@ -272,8 +301,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         if (pre) return pre_len[(hd.it - bx) / G];
         return p.log_len ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
     };
-    auto resolve_slot = [&](Head &hd, int it, int s) {
+    auto resolve_slot = [&](Head &hd, int it, int s, int half) {
         hd.it = it;
+        hd.half = half;
         hd.s = s;
         hd.ok = 0;
         hd.c = 0;
@@ -301,7 +331,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         const bool merge = p.eager || (p.auto_merge && c >= p.L - 1);
         hd.mk = !merge ? MK_APPEND : c > TM_ENT ? MK_ROUNDS : DELTA ? MK_PASS2 : MK_FUSED;
         hd.nl = (c + EPC - 1) / EPC;
-        hd.n = hd.nl + NCH + (hd.mk == MK_PASS2 ? NCH : 0);
+        hd.n = hd.nl + (hd.half ? NCH / 2 : NCH) + (hd.mk == MK_PASS2 ? NCH : 0);
     };
     // L2 warm-up of a head's token rows (they depend on the work item only)
     auto warm_token = [&](int it) {
@@ -323,10 +353,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     Head cur, nxt;
     nxt.ok = 0;
     nxt.n = 0;
-    const int it0 = item_at(w);
+    int half0 = 0, half_nxt = 0;
+    const int it0 = item_at(w, half0);
     warm_token(it0);
-    resolve_slot(cur, it0, slot_of(it0));
-    int it_nxt = grab();                 // the warp's next head, and its slot id, one head early
+    resolve_slot(cur, it0, slot_of(it0), half0);
+    int it_nxt = grab(half_nxt);         // the warp's next head, and its slot id, one head early
     int s_nxt = slot_of(it_nxt);
     bool nxt_res = false;                // nxt's live length known
     int c_nxt = 0;
@@ -347,7 +378,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     ptx::bulk_g2s(dst + (size_t)(i - lo) * ESF, src + (size_t)i * E, ESB, bar, pol_stream);
             }
         } else {
-            const int y = x - hd.nl;
+            const int y = x - hd.nl + (hd.half == 2 ? NCH / 2 : 0);   // the upper half starts at row 64
             const bool keep = y < NCH && (hd.mk == MK_PASS2 || hd.mk == MK_ROUNDS);
             ptx::mbar_arrive_expect_tx(bar, CB);
             ptx::bulk_g2s(dst, p.state + hd.head * (size_t)(DK * DV) + (size_t)(y & (NCH - 1)) * CF, CB, bar,
@@ -406,7 +437,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     while (cur.it < n_items) {
         // the next head: slot id read one head ago; its live length is loaded now
         // and used when the stream reaches it
-        resolve_slot(nxt, it_nxt, s_nxt);
+        resolve_slot(nxt, it_nxt, s_nxt, half_nxt);
         nxt_res = false;
         c_nxt = len_of(nxt);
         if (nxt.ok) warm_token(nxt.it);
@@ -537,6 +568,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
             if (abort) break;
             if (stage_tm) ptx::tmem_wait_st();
+            if (cur.half == 2) Yq = make_float4(0.f, 0.f, 0.f, 0.f);  // counted once, by the lower half
 
             // new rows of one 16-row block of the merged state from its Sbar rows in
             // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending.
@@ -597,7 +629,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             // -- AppendDecode pass 1: y_q = Sbar^T qt, y_k = Sbar^T kt (columns 4l..4l+3);
             //    without the delta rule a merge writes its new rows here as well
             const float4 v4 = make_float4(v_own[0], v_own[1], v_own[2], v_own[3]);
-            for (int cx = 0; cx < NCH; ++cx) {
+            const int cx0 = cur.half == 2 ? NCH / 2 : 0, cx1 = cur.half == 1 ? NCH / 2 : NCH;
+            for (int cx = cx0; cx < cx1; ++cx) {
                 if (!wait_chunk()) { abort = true; break; }
                 const float *sb = st + (size_t)(gc % NSW) * CF;
 #pragma unroll
@@ -632,8 +665,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                 o[x] = fmaf(bt[x], kq, yq[x]);
             }
             const float4 bt4 = make_float4(bt[0], bt[1], bt[2], bt[3]);
-            if (p.want_out)
+            bool commits = true;  // this work item finalizes the head
+            if (cur.half) {
+                // Split merge: the first half to finish leaves its partial (its rows'
+                // share of Sbar^T qt; the lower half also the replay) in out and marks
+                // it; the second adds it to its own and the token term, and commits.
+                float4 *orow = reinterpret_cast<float4 *>(p.out + row * DV) + lane;
+                int *cm = comb + (cur.it - bx) / G;
+                int first = 0;
+                if (lane == 0) first = atomicAdd(cm, 1);
+                first = __shfl_sync(FULL, first, 0);
+                if (first == 0) {
+                    *orow = Yq;
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicAdd(cm, 4);  // partial ready (arrivals count 1, 2)
+                    commits = false;
+                } else {
+                    // the other half is past its atomic and stores its partial next
+                    bool ready = false;
+                    if (lane == 0) {
+                        const uint64_t t0 = ptx::globaltimer_ns();
+                        while (!(ready = (atomicAdd(cm, 0) & 4) != 0)) {
+                            if (ptx::globaltimer_ns() - t0 > WAIT_NS) break;
+                        }
+                    }
+                    ready = __shfl_sync(FULL, ready ? 1 : 0, 0) != 0;
+                    if (!ready) { abort = true; break; }
+                    __threadfence();
+                    const float4 other = __ldcg(orow);
+                    *orow = make_float4(o[0] + other.x, o[1] + other.y, o[2] + other.z, o[3] + other.w);
+                }
+            } else if (p.want_out) {
                 *reinterpret_cast<float4 *>(p.out + row * DV + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+            }
             if (mk == MK_APPEND) {
                 float *ent = ring + (size_t)c * E;
                 put_seg4<LC::B16>(ent + BO, lane, bt4);
@@ -758,7 +823,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
             // -- Finalize: the last unit of the (slot, layer) commits the live length
             //    (the atomic is issued now, its result looked at one head later)
-            if (!p.eager) {
+            if (!p.eager && commits) {
                 if (lane == 0) fin_old = atomicAdd(p.arrive + sl, 1);
                 fin_sl = sl;
                 fin_len = mk != MK_APPEND ? 0 : c + 1;
@@ -774,7 +839,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         cur = nxt;
         nxt.ok = 0;
         nxt.n = 0;
-        it_nxt = grab();
+        it_nxt = grab(half_nxt);
         s_nxt = slot_of(it_nxt);
         nxt_res = false;
         issue_upto(gc + NSW);

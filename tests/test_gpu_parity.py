@@ -401,3 +401,25 @@ def test_cluster_replay_matches_per_tile_bit_for_bit(name, tile_v):
     for layer in res["cluster"][0]:
         np.testing.assert_array_equal(res["cluster"][0][layer], res["per_tile"][0][layer])
         np.testing.assert_array_equal(res["cluster"][1][layer], res["per_tile"][1][layer])
+
+
+# ---- merge heads split in two halves (CTAs with more heads than warps) ---------------
+@pytest.mark.parametrize("staggered,log_format", [(False, "fp32"), (True, "fp32"), (True, "compact")])
+def test_split_merge_heads_match_the_oracle(staggered, log_format):
+    """3200 heads over at most 148 CTAs: every CTA orders its heads and splits each merge
+    without the delta rule into two half-tile work items whose partial outputs combine.
+    Non-staggered, every slot merges at once (all heads split); staggered, a few do."""
+    wl = synth.GLA_DIAG.with_(batch=200, steps=24, log_cap=4, staggered=staggered)
+    rows = np.array([0, 77, 199])
+    r = DecodeRunner(wl, tile_v=128, log_format=log_format)
+    T = wl.steps
+    outs, states, kept = H.gpu_rollout(r, T, ckpts=[T], keep_inputs=True)
+    assert r.errors() == 0
+    O, S = H.oracle_reference(wl, 0, T, rows=rows, ckpts=[T], main_inputs=kept[0])
+    H.check_steps(outs[0][:, rows], O)
+    H.check_steps(states[0][:, rows], S, elem=None, what="state")
+    # against the in-library eager step over every row
+    re_ = DecodeRunner(wl, mode="eager", tile_v=16)
+    oe, se, _ = H.gpu_rollout(re_, T, ckpts=[T])
+    H.check_steps(outs[0], oe[0], tol=H.REL_L2_GPU, elem=None, what="deferred vs eager")
+    H.check_steps(states[0], se[0], tol=H.REL_L2_GPU, elem=None, what="state")
