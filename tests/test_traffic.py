@@ -32,3 +32,20 @@ def test_entry_and_token_sizes():
     # GVA: q and k shared by two value heads
     assert traffic.token_bytes(synth.GDN_GVA) == 2 * 128 * 2 / 2 + 256 + 4 + 4 + 512
     assert traffic.deferred_head_step(synth.KDA, 0, True) == traffic.eager_head_step(synth.KDA)
+
+
+def test_compact_entry_bytes_agree_with_the_library_layout():
+    """The byte model's compact entry (the bytes that must move) against the library's
+    row size (dl_log_bytes): equal, except that scalar decay pads Lambda_0 to 16 B."""
+    import ctypes
+    from recurrent_state_serving_b200 import deltalog as dl
+    for decay in ("none", "scalar", "diag"):
+        for update in ("add", "delta"):
+            wl = synth.GLA_DIAG.with_(decay=decay, update=update)
+            d = dl.dl_pool_desc(1, 1, 1, 1, wl.d_k, wl.d_v, 1, dl.DECAY[decay], dl.UPDATE[update], 0,
+                                dl.LOG_FORMAT["compact"], 0)
+            n = ctypes.c_int64()
+            assert dl.library().dl_log_bytes(ctypes.byref(d), ctypes.byref(n)) == dl.DL_OK
+            pad = 12 if decay == "scalar" else 0
+            assert traffic.entry_bytes(wl, "compact") + pad == n.value
+            assert traffic.entry_bytes(wl, "compact") < traffic.entry_bytes(wl)
