@@ -21,6 +21,7 @@ from dataclasses import dataclass
 import torch
 
 from . import deltalog as dl
+from . import tuning
 
 
 class SlotAllocator:
@@ -70,12 +71,19 @@ class DecodeServer:
     Inputs of a step are given per layer as dicts of device tensors with one row per
     active request, in the order of ``active`` (q, k: [B, H_k, d_k]; v: [B, H, d_v];
     lam: [B, H] / [B, H, d_k] or per-head constants; beta: [B, H]).
+
+    ``log_cap="auto"`` takes the merge interval with the fewest modelled HBM bytes per
+    head-step for this operator's shape, decay, update rule and log layout
+    (``tuning.auto_log_cap``), which is the right choice when the batch fills the GPU.
     """
 
     def __init__(self, *, n_slots, n_layers, n_heads, d_k, d_v, log_cap, decay="none",
                  update="add", n_kheads=None, in_dtype=torch.bfloat16, lambda_per_head=False,
                  log_format="fp32", tile_v=0, max_batch=None, device="cuda", use_graphs=True):
-        self.pool = dl.Pool(n_slots, n_layers, n_heads, d_k, d_v, log_cap, decay=decay,
+        if log_cap == "auto":
+            log_cap = tuning.auto_log_cap(d_k, d_v, decay, update, log_format)
+        self.log_cap = int(log_cap)
+        self.pool = dl.Pool(n_slots, n_layers, n_heads, d_k, d_v, self.log_cap, decay=decay,
                             update=update, n_kheads=n_kheads, device=device, log_format=log_format,
                             tile_v=tile_v)
         self.alloc = SlotAllocator(n_slots)
