@@ -58,6 +58,19 @@ def test_modelled_pick_agrees_with_the_measured_sweep():
     assert tuning.modelled_log_cap(synth.GLA_DIAG, measured) == 8
 
 
+def test_modelled_pick_agrees_with_the_retnet_sweep():
+    # RetNet scalar decay, 8 layers, B = 256, H = 32, staggered merges: decode
+    # head-steps/s on one B200 per interval and log layout (CUDA graph of 512 steps)
+    fp32 = {8: 71.36e6, 16: 71.61e6, 32: 65.46e6}
+    compact = {8: 72.77e6, 16: 75.86e6, 32: 71.76e6}
+    wl = synth.RETNET.with_(batch=256)
+    assert tuning.modelled_log_cap(wl, compact, "compact") == tuning.select_log_cap(compact) == 16
+    # fp32: the model has L = 8 and 16 within 0.1 % of each other; so do the measurements
+    assert tuning.modelled_log_cap(wl, fp32) == 8
+    assert abs(fp32[8] / fp32[16] - 1) < 0.005
+    assert tuning.cycle_bytes(wl, 16) / tuning.cycle_bytes(wl, 8) - 1 < 0.002
+
+
 def test_select_from_measurements():
     assert tuning.select_log_cap({4: 1.0, 8: 3.0, 16: 2.0}) == 8
     # times: lower is better
