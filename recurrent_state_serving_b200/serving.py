@@ -123,10 +123,10 @@ class DecodeServer:
         dense base of a free slot, whose log is reset.  Returns the request id."""
         if len(self.active) >= self.max_batch:
             raise RuntimeError("batch is full")
-        s = self.alloc.alloc()
         want = (self.n_layers, self.H, self.d_k, self.d_v)
         if tuple(prefill_state.shape) != want:
             raise ValueError(f"prefill state must be {list(want)}")
+        s = self.alloc.alloc()
         self.pool.state[s].copy_(prefill_state.to(self.device, torch.float32))
         dl.dl_reset_slots(self.pool, torch.tensor([s], dtype=torch.int32, device=self.device))
         rid = self._next_rid
@@ -176,6 +176,24 @@ class DecodeServer:
             if st != dl.DL_OK:
                 raise dl.DeltaLogError(st, "dl_decode_step")
 
+    def _check_inputs(self, inputs, B: int):
+        """Every input the server's operator needs, for every layer, with exactly the
+        rows of the active requests (no broadcasting into the step buffers)."""
+        if len(inputs) != self.n_layers:
+            raise ValueError(f"expected inputs for {self.n_layers} layers, got {len(inputs)}")
+        for l, x in enumerate(inputs):
+            b = self.bufs[l]
+            for key in ("q", "k", "v", "lam", "beta"):
+                if b[key] is None:
+                    if x.get(key) is not None:
+                        raise ValueError(f"layer {l}: this server takes no '{key}' per step")
+                    continue
+                if x.get(key) is None:
+                    raise ValueError(f"layer {l}: '{key}' is missing")
+                want = tuple(b[key][:B].shape)
+                if tuple(x[key].shape) != want:
+                    raise ValueError(f"layer {l}: '{key}' must be {list(want)}, got {list(x[key].shape)}")
+
     def step(self, inputs) -> list[torch.Tensor]:
         """One decode step of every active request over all layers.  ``inputs[l]`` holds
         layer l's rows.  Returns each layer's outputs [B, H, d_v] (views of the server's
@@ -183,10 +201,11 @@ class DecodeServer:
         B = len(self.active)
         if B == 0:
             return []
+        self._check_inputs(inputs, B)
         for l, x in enumerate(inputs):
             b = self.bufs[l]
             for key in ("q", "k", "v", "lam", "beta"):
-                if b.get(key) is not None and x.get(key) is not None:
+                if b[key] is not None:
                     b[key][:B].copy_(x[key], non_blocking=True)
         if self.use_graphs:
             g = self._graphs.get(B)

@@ -27,6 +27,49 @@ def test_slot_allocator_reuses_the_lowest_free_slot():
         SlotAllocator(0)
 
 
+def _host_server(**kw):
+    # the pool's buffers are host tensors here: only the host-side checks run
+    import torch
+    from recurrent_state_serving_b200.serving import DecodeServer
+    args = dict(n_slots=3, n_layers=2, n_heads=4, n_kheads=2, d_k=16, d_v=16, log_cap=4,
+                decay="diag", update="delta", device="cpu", use_graphs=False)
+    args.update(kw)
+    return DecodeServer(**args), torch
+
+
+def test_server_rejects_a_bad_prefill_without_taking_a_slot():
+    srv, torch = _host_server()
+    with pytest.raises(ValueError):
+        srv.admit(torch.zeros(2, 4, 16, 8))
+    assert srv.alloc.n_free == 3 and srv.active == []
+
+
+def test_server_checks_every_step_input():
+    srv, torch = _host_server()
+    B = 2
+
+    def layer(**over):
+        x = {"q": torch.zeros(B, 2, 16), "k": torch.zeros(B, 2, 16), "v": torch.zeros(B, 4, 16),
+             "lam": torch.zeros(B, 4, 16), "beta": torch.zeros(B, 4)}
+        x.update(over)
+        return x
+
+    srv._check_inputs([layer(), layer()], B)
+    with pytest.raises(ValueError, match="layers"):
+        srv._check_inputs([layer()], B)
+    with pytest.raises(ValueError, match="'beta' is missing"):
+        srv._check_inputs([layer(), layer(beta=None)], B)
+    # a per-head row would broadcast over the batch: refused
+    with pytest.raises(ValueError, match="'lam' must be"):
+        srv._check_inputs([layer(lam=torch.zeros(4, 16)), layer()], B)
+    with pytest.raises(ValueError, match="'v' must be"):
+        srv._check_inputs([layer(v=torch.zeros(B + 1, 4, 16)), layer()], B)
+    add, _ = _host_server(update="add", decay="none")
+    with pytest.raises(ValueError, match="no 'beta'"):
+        add._check_inputs([layer(lam=None), layer(lam=None)], B)
+    add._check_inputs([layer(lam=None, beta=None), layer(lam=None, beta=None)], B)
+
+
 # -- GPU: a request schedule over 30 steps ---------------------------------------
 L_LAYERS, H, HK, D, LOG_CAP = 2, 4, 2, 128, 5
 # (step, action, request index): admissions and retirements
