@@ -108,11 +108,16 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _dev_tensor(t, name, dtype=None):
+def _dev_tensor(t, name, dtype=None, device=None):
+    """A contiguous CUDA tensor of the given dtype, on the pool's device when one is
+    given (the library sees only the pointer, so a tensor of another GPU would be
+    read through the wrong context)."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the pool on {device}")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -166,15 +171,16 @@ class Pool:
 
 
 def _step_args(pool, slots, q, k, v, lam, beta, out, lambda_per_head):
-    slots = _dev_tensor(slots, "slots", torch.int32)
-    q = _dev_tensor(q, "q")
-    k = _dev_tensor(k, "k", q.dtype)
-    v = _dev_tensor(v, "v", q.dtype)
+    dev = pool.state.device
+    slots = _dev_tensor(slots, "slots", torch.int32, dev)
+    q = _dev_tensor(q, "q", None, dev)
+    k = _dev_tensor(k, "k", q.dtype, dev)
+    v = _dev_tensor(v, "v", q.dtype, dev)
     if q.dtype not in DTYPE:
         raise TypeError("q/k/v must be float32 or bfloat16")
-    lam = _dev_tensor(lam, "lambda", torch.float32)
-    beta = _dev_tensor(beta, "beta", torch.float32)
-    out = _dev_tensor(out, "out", torch.float32)
+    lam = _dev_tensor(lam, "lambda", torch.float32, dev)
+    beta = _dev_tensor(beta, "beta", torch.float32, dev)
+    out = _dev_tensor(out, "out", torch.float32, dev)
     B = slots.numel()
     if q.shape != (B, pool.n_kheads, pool.d_k) or k.shape != q.shape:
         raise ValueError(f"q/k must be [{B}, {pool.n_kheads}, {pool.d_k}]")
@@ -242,24 +248,27 @@ def dl_eager_step(pool: Pool, layer: int, slots, q, k, v, lam=None, beta=None, o
 
 
 def dl_merge(pool: Pool, layer: int, slots, stream=None):
-    slots = _dev_tensor(slots, "slots", torch.int32)
+    slots = _dev_tensor(slots, "slots", torch.int32, pool.state.device)
     _check(_lib.dl_merge(pool.handle, layer, _ptr(slots), slots.numel(), _stream(stream)),
            "dl_merge")
 
 
 def dl_materialize(pool: Pool, layer: int, slots, dense_out=None, stream=None):
-    slots = _dev_tensor(slots, "slots", torch.int32)
+    dev = pool.state.device
+    slots = _dev_tensor(slots, "slots", torch.int32, dev)
+    want = (slots.numel(), pool.n_heads, pool.d_k, pool.d_v)
     if dense_out is None:
-        dense_out = torch.empty(slots.numel(), pool.n_heads, pool.d_k, pool.d_v,
-                                dtype=torch.float32, device=pool.state.device)
-    dense_out = _dev_tensor(dense_out, "dense_out", torch.float32)
+        dense_out = torch.empty(want, dtype=torch.float32, device=dev)
+    dense_out = _dev_tensor(dense_out, "dense_out", torch.float32, dev)
+    if tuple(dense_out.shape) != want:
+        raise ValueError(f"dense_out must be {list(want)}, got {list(dense_out.shape)}")
     _check(_lib.dl_materialize(pool.handle, layer, _ptr(slots), slots.numel(), _ptr(dense_out),
                                _stream(stream)), "dl_materialize")
     return dense_out
 
 
 def dl_reset_slots(pool: Pool, slots, stream=None):
-    slots = _dev_tensor(slots, "slots", torch.int32)
+    slots = _dev_tensor(slots, "slots", torch.int32, pool.state.device)
     _check(_lib.dl_reset_slots(pool.handle, _ptr(slots), slots.numel(), _stream(stream)),
            "dl_reset_slots")
 

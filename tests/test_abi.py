@@ -5,6 +5,7 @@ import ctypes
 import subprocess
 
 import pytest
+import torch
 
 from recurrent_state_serving_b200 import deltalog as dl
 
@@ -211,3 +212,46 @@ def test_compact_log_needs_bf16_inputs():
     d = _desc(log_format=1, arrive=None)
     assert lib.dl_decode_step_noalloc(ctypes.byref(d), 0, ctypes.byref(a), 1, None) == dl.DL_ERR_DTYPE
     lib.dl_destroy_pool(h)
+
+
+class _ReportsCuda(torch.Tensor):
+    """A host tensor that passes the binding's CUDA-tensor test, so that its later
+    checks (device, shape) can be exercised without a GPU.  Every case below is
+    refused before any library call."""
+    @property
+    def is_cuda(self):
+        return True
+
+
+def _rc(t):
+    return torch.Tensor._make_subclass(_ReportsCuda, t)
+
+
+def test_binding_checks_shapes_and_device_before_the_library():
+    pool = dl.Pool(3, 1, 2, 16, 16, 4, decay="diag", update="delta", device="cpu")
+    slots = _rc(torch.zeros(2, dtype=torch.int32))
+    # materialize: the output buffer must be exactly [B, H, d_k, d_v]
+    with pytest.raises(ValueError, match="dense_out must be"):
+        dl.dl_materialize(pool, 0, slots, dense_out=_rc(torch.zeros(2, 2, 16, 17)))
+    with pytest.raises(ValueError, match="dense_out must be"):
+        dl.dl_materialize(pool, 0, slots, dense_out=_rc(torch.zeros(1, 2, 16, 16)))
+    # tensors on another device than the pool's
+    other = _rc(torch.zeros(2, dtype=torch.int32, device="meta"))
+    for fn in (lambda s: dl.dl_materialize(pool, 0, s), lambda s: dl.dl_merge(pool, 0, s),
+               lambda s: dl.dl_reset_slots(pool, s)):
+        with pytest.raises(ValueError, match="is on meta"):
+            fn(other)
+    q = _rc(torch.zeros(2, 2, 16))
+    v = _rc(torch.zeros(2, 2, 16))
+    lam = _rc(torch.zeros(2, 2, 16))
+    beta = _rc(torch.zeros(2, 2))
+    out = _rc(torch.zeros(2, 2, 16))
+    with pytest.raises(ValueError, match="is on meta"):
+        dl.dl_decode_step(pool, 0, slots, q, q, v, lam=lam, beta=_rc(torch.zeros(2, 2, device="meta")),
+                          out=out)
+    with pytest.raises(ValueError, match="lambda must be"):
+        dl.dl_decode_step(pool, 0, slots, q, q, v, lam=_rc(torch.zeros(2, 2)), beta=beta, out=out)
+    with pytest.raises(ValueError, match="out must be"):
+        dl.dl_decode_step(pool, 0, slots, q, q, v, lam=lam, beta=beta, out=_rc(torch.zeros(2, 2, 8)))
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        dl.dl_decode_step(pool, 0, slots, torch.zeros(2, 2, 16), q, v, lam=lam, beta=beta, out=out)
