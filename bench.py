@@ -579,7 +579,10 @@ def run_reference(a, wl):
     value = units * a.steps / sum(times)
     sample = (f"{units} of {wl.units_per_step} head-steps per step ({n_rows} slots x {wl.n_heads} heads, "
               f"layer 0), fp64 eager oracle advanced one token per step")
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+    # n_gpus echoes the launch (the arm is run with the same --gpus N as ours); the
+    # oracle itself runs on the host cores of rank 0 and uses no GPU
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+            "device": f"host CPU, {threads} threads (no GPU)",
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch, a.log_format, a.replay),
