@@ -84,6 +84,8 @@ def parse():
                     help="rotate mode: replay the timed steps from a CUDA graph or launch them directly")
     ap.add_argument("--replay", default="per_tile", choices=["per_tile", "cluster"],
                     help="value-tiled kernel: ReplayPrep formed per tile, or shared by a head's tiles as one cluster")
+    ap.add_argument("--e2e-copies", default="per_tensor", choices=["per_tensor", "packed"],
+                    help="end-to-end leg: copy each input/output tensor, or one packed buffer per step")
     ap.add_argument("--log-format", default="fp32", choices=["fp32", "compact"],
                     help="log entry layout: fp32 [a|b|Lambda], or compact (bf16 a, bf16 b without the delta rule)")
     return ap.parse_args()
@@ -306,6 +308,52 @@ def graph_upload(graph, stream) -> bool:
 # ---------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------
+PACK_ALIGN = 256
+
+
+def pack_layout(spec, align: int = PACK_ALIGN):
+    """Byte offsets of a step's tensors packed into one buffer.
+
+    spec: one dict per layer, {name: (shape, dtype) or None}.  Each tensor starts on
+    an ``align``-byte boundary.  Returns (total bytes, one {name: offset or None}
+    dict per layer)."""
+    off, offs = 0, []
+    for layer in spec:
+        d = {}
+        for k, v in layer.items():
+            if v is None:
+                d[k] = None
+                continue
+            shape, dtype = v
+            n = int(np.prod(shape)) * torch_elem_size(dtype)
+            off = -(-off // align) * align
+            d[k] = off
+            off += n
+        offs.append(d)
+    return -(-off // align) * align, offs
+
+
+def torch_elem_size(dtype) -> int:
+    import torch
+    return torch.empty((), dtype=dtype).element_size()
+
+
+def packed_views(buf, spec, offs):
+    """Typed views of a uint8 buffer laid out by pack_layout."""
+    out = []
+    for layer, o in zip(spec, offs):
+        d = {}
+        for k, v in layer.items():
+            if v is None:
+                d[k] = None
+                continue
+            shape, dtype = v
+            n = int(np.prod(shape)) * torch_elem_size(dtype)
+            d[k] = buf[o[k]:o[k] + n].view(dtype).view(shape)
+        out.append(d)
+    return out
+
+
 def run_gpu(a, wl, rank, world, dist):
     import torch
     from recurrent_state_serving_b200 import deltalog as dl
@@ -468,35 +516,68 @@ def run_gpu(a, wl, rank, world, dist):
 
     # ---- end to end through the public API with host buffers ----
     if not a.no_e2e:
-        pin = lambda t: None if t is None else t.cpu().pin_memory()
-        host_dev = [[{k: pin(v) for k, v in x.items()} for x in per_layer] for per_layer in dev_inputs]
-        h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
-        d2h = sum(o.numel() * o.element_size() for o in outs)
-        # two sets of device staging buffers, outputs and pinned host outputs; the
-        # serial form uses set 0 only
-        stage = [[{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
-                  for x in dev_inputs[0]] for _ in range(2)]
-        outs_e = [[torch.empty_like(o) for o in outs] for _ in range(2)]
-        out_host = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
+        # Inputs and outputs are double-buffered (set j % 2 for step j); the serial
+        # form uses set 0 only.  --e2e-copies packed lays each step's inputs (all
+        # layers) out in one pinned host buffer and every layer's output in one device
+        # buffer, so a step is one upload and one download; per_tensor copies each
+        # input and output tensor on its own.
+        if a.e2e_copies == "packed":
+            spec = [{k: (None if v is None else (tuple(v.shape), v.dtype)) for k, v in x.items()}
+                    for x in dev_inputs[0]]
+            in_bytes, in_offs = pack_layout(spec)
+            host_pk = []
+            for per_layer in dev_inputs:
+                hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+                for view, x in zip(packed_views(hb, spec, in_offs), per_layer):
+                    for k, v in x.items():
+                        if v is not None:
+                            view[k].copy_(v.cpu())
+                host_pk.append(hb)
+            out_spec = [{"o": (tuple(o.shape), o.dtype)} for o in outs]
+            out_bytes, out_offs = pack_layout(out_spec)
+            h2d, d2h = in_bytes, out_bytes   # the buffers copied (tensors plus alignment padding)
+            stage_buf = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+            stage = [packed_views(sb, spec, in_offs) for sb in stage_buf]
+            out_buf = [torch.empty(out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+            outs_e = [[v["o"] for v in packed_views(ob, out_spec, out_offs)] for ob in out_buf]
+            out_host = [torch.empty(out_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+
+            def upload(t, b):
+                stage_buf[b].copy_(host_pk[t], non_blocking=True)
+
+            def download(b):
+                out_host[b].copy_(out_buf[b], non_blocking=True)
+        else:
+            pin = lambda t: None if t is None else t.cpu().pin_memory()
+            host_dev = [[{k: pin(v) for k, v in x.items()} for x in per_layer] for per_layer in dev_inputs]
+            h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
+            d2h = sum(o.numel() * o.element_size() for o in outs)
+            stage = [[{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
+                      for x in dev_inputs[0]] for _ in range(2)]
+            outs_e = [[torch.empty_like(o) for o in outs] for _ in range(2)]
+            out_host = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
+
+            def upload(t, b):
+                for l in range(wl.n_layers):
+                    for k, v in host_dev[t][l].items():
+                        if v is not None:
+                            stage[b][l][k].copy_(v, non_blocking=True)
+
+            def download(b):
+                for l in range(wl.n_layers):
+                    out_host[b][l].copy_(outs_e[b][l], non_blocking=True)
         prep_2 = [[[dl.PreparedStep("decode", r.pool, l, gs, s_["q"], s_["k"], s_["v"], s_["lam"],
                                     s_["beta"], outs_e[b][l], wl.lambda_const) for l, s_ in enumerate(stage[b])]
                    for b in range(2)] for gs in r.group_slots]
-
-        def upload(src, b):
-            for l in range(wl.n_layers):
-                for k, v in src[l].items():
-                    if v is not None:
-                        stage[b][l][k].copy_(v, non_blocking=True)
-
-        def download(b):
-            for l in range(wl.n_layers):
-                out_host[b][l].copy_(outs_e[b][l], non_blocking=True)
+        copies = ("one H2D copy of the step's packed pinned inputs" if a.e2e_copies == "packed"
+                  else "H2D copies of the step's pinned inputs")
+        copies_out = "one D2H copy of every layer's o_t" if a.e2e_copies == "packed" else "D2H of o_t"
 
         def serial_calls(j):
-            src, prep = host_dev[j % ndist], prep_2[j % R][0]
+            t, prep = j % ndist, prep_2[j % R][0]
 
             def one():
-                upload(src, 0)
+                upload(t, 0)
                 for p_ in prep:
                     check(p_())
                 download(0)
@@ -515,7 +596,7 @@ def run_gpu(a, wl, rank, world, dist):
         last = W + K - 1
 
         def piped_calls(j):
-            src, b = host_dev[j % ndist], j % 2
+            t, b = j % ndist, j % 2
             prep = prep_2[j % R][b]
 
             def one():
@@ -526,7 +607,7 @@ def run_gpu(a, wl, rank, world, dist):
                     s_out.wait_stream(comp)
                 s_in.wait_event(ev_comp[b])
                 with torch.cuda.stream(s_in):
-                    upload(src, b)
+                    upload(t, b)
                 ev_in[b].record(s_in)
                 comp.wait_event(ev_in[b])
                 comp.wait_event(ev_out[b])
@@ -547,18 +628,20 @@ def run_gpu(a, wl, rank, world, dist):
         tot_s = reduce_max(ms_s)
         serial = {"value": whole_job_rate(wl.units_per_step * K, world, tot_s), "unit": UNIT,
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_s / K,
-                  "path": "one stream: pinned host inputs -> H2D copy -> dl_decode_step per layer -> "
-                          "D2H of o_t, step after step, all inside the events"}
+                  "copies": a.e2e_copies,
+                  "path": f"one stream: {copies} -> dl_decode_step per layer -> {copies_out}, "
+                          "step after step, all inside the events"}
         if a.l2 == "rotate":
             ms_p = timed(piped_calls, K, graph_ok=False)
             assert r.errors() == 0
             tot_p = reduce_max(ms_p)
             result["e2e"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_p), "unit": UNIT,
                              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_p / K,
-                             "path": "pinned host inputs -> H2D copy (copy stream) -> dl_decode_step per "
-                                     "layer (compute stream) -> D2H of o_t (second copy stream), double-"
-                                     "buffered so that step j+1's upload and step j-1's download overlap "
-                                     "step j's kernels; every copy inside the events"}
+                             "copies": a.e2e_copies,
+                             "path": f"{copies} (copy stream) -> dl_decode_step per layer (compute "
+                                     f"stream) -> {copies_out} (second copy stream), double-buffered so "
+                                     "that step j+1's upload and step j-1's download overlap step j's "
+                                     "kernels; every copy inside the events"}
             result["e2e_serial"] = serial
         else:
             result["e2e"] = serial

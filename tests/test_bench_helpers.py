@@ -2,6 +2,7 @@
 and the byte accounting of the timed launches."""
 import os
 
+import numpy as np
 import pytest
 
 import bench
@@ -77,3 +78,78 @@ def test_live_entries_follow_each_group_cycle():
         seen[g] += 1
     # one group: the plain per-step cycle
     np.testing.assert_array_equal(bench.live_entries(offs, 13, 1, L), (offs + 13) % L)
+
+
+def _step_spec(wl):
+    import torch
+    bf = torch.bfloat16 if wl.in_dtype == "bf16" else torch.float32
+    x = synth.step_inputs(wl.with_(batch=3), 0, 0)
+    spec = []
+    for _ in range(wl.n_layers):
+        d = {}
+        for k, v in x.items():
+            d[k] = None if v is None else (tuple(v.shape), bf if k in ("q", "k", "v") else torch.float32)
+        spec.append(d)
+    return spec
+
+
+@pytest.mark.parametrize("wl", [synth.GLA_DIAG, synth.KDA.with_(n_layers=3), synth.RETNET.with_(n_layers=2),
+                                synth.GDN_GVA, synth.TINY_LA], ids=lambda w: w.name)
+def test_packed_step_inputs(wl):
+    """One buffer per step: every tensor on a 256-byte boundary, no overlaps, the
+    views round-trip the values, and the binding takes them as they are."""
+    import torch
+    from recurrent_state_serving_b200 import deltalog as dl
+    spec = _step_spec(wl)
+    total, offs = bench.pack_layout(spec)
+    assert total % bench.PACK_ALIGN == 0
+    spans = []
+    for layer, o in zip(spec, offs):
+        for k, v in layer.items():
+            if v is None:
+                assert o[k] is None
+                continue
+            n = int(np.prod(v[0])) * bench.torch_elem_size(v[1])
+            assert o[k] % bench.PACK_ALIGN == 0
+            spans.append((o[k], o[k] + n))
+    spans.sort()
+    assert all(a1 <= b0 for (_, a1), (b0, _) in zip(spans, spans[1:]))
+    assert spans[-1][1] <= total
+    padding = total - sum(b - a for a, b in spans)
+    assert 0 <= padding < bench.PACK_ALIGN * (len(spans) + 1)
+
+    buf = torch.zeros(total, dtype=torch.uint8)
+    views = bench.packed_views(buf, spec, offs)
+    g = torch.Generator().manual_seed(5)
+    vals = []
+    for layer in views:
+        d = {}
+        for k, v in layer.items():
+            if v is not None:
+                assert v.is_contiguous() and v.data_ptr() % bench.PACK_ALIGN == buf.data_ptr() % bench.PACK_ALIGN
+                d[k] = torch.randn(v.shape, generator=g).to(v.dtype)
+                v.copy_(d[k])
+        vals.append(d)
+    again = bench.packed_views(buf.clone(), spec, offs)
+    for d, layer in zip(vals, again):
+        for k, v in d.items():
+            assert torch.equal(layer[k], v)
+
+    # the binding accepts the views and passes their own addresses (no copies)
+    class _RC(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+    rc = lambda t: None if t is None else torch.Tensor._make_subclass(_RC, t)
+    B = 3
+    pool = dl.Pool(B, wl.n_layers, wl.n_heads, wl.d_k, wl.d_v, 4, decay=wl.decay, update=wl.update,
+                   n_kheads=wl.n_kheads, device="cpu")
+    out_spec = [{"o": ((B, wl.n_heads, wl.d_v), torch.float32)} for _ in range(wl.n_layers)]
+    ob, oo = bench.pack_layout(out_spec)
+    outs = bench.packed_views(torch.zeros(ob, dtype=torch.uint8), out_spec, oo)
+    slots = rc(torch.arange(B, dtype=torch.int32))
+    for layer, o in zip(views, outs):
+        a = dl._step_args(pool, slots, rc(layer["q"]), rc(layer["k"]), rc(layer["v"]), rc(layer["lam"]),
+                          rc(layer["beta"]), rc(o["o"]), wl.lambda_const)
+        assert a.q == layer["q"].data_ptr() and a.v == layer["v"].data_ptr()
+        assert a.out == o["o"].data_ptr()
