@@ -255,3 +255,30 @@ def test_binding_checks_shapes_and_device_before_the_library():
         dl.dl_decode_step(pool, 0, slots, q, q, v, lam=lam, beta=beta, out=_rc(torch.zeros(2, 2, 8)))
     with pytest.raises(TypeError, match="CUDA tensor"):
         dl.dl_decode_step(pool, 0, slots, torch.zeros(2, 2, 16), q, v, lam=lam, beta=beta, out=out)
+
+
+def test_header_compiles_as_c99_and_matches_the_binding(tmp_path):
+    """A plain C consumer of include/deltalog.h: it must build with a C compiler in
+    strict mode, link against the library, get the documented results from the
+    calls that need no GPU, and see the same struct layouts as the ctypes binding."""
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(dl.LIB_PATH)
+    exe = str(tmp_path / "c_abi_consumer")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"), os.path.join(root, "tests", "c_abi_consumer.c"),
+                    "-o", exe, "-L", libdir, "-ldeltalog", f"-Wl,-rpath,{libdir}"], check=True)
+    run = subprocess.run([exe], capture_output=True, text=True)
+    assert run.returncode == 0, run.stdout + run.stderr
+    seen = dict(line.rsplit(" ", 1) for line in run.stdout.splitlines() if " " in line)
+    assert seen["sizeof.dl_pool_desc"] == str(ctypes.sizeof(dl.dl_pool_desc))
+    assert seen["sizeof.dl_step_args"] == str(ctypes.sizeof(dl.dl_step_args))
+    n = 0
+    for key, off in seen.items():
+        struct, _, field = key.partition(".")
+        if struct in ("dl_pool_desc", "dl_step_args"):
+            cls = getattr(dl, struct)
+            assert getattr(cls, "lambda_" if field == "lambda" else field).offset == int(off), key
+            n += 1
+    assert n == 22
+    assert run.stdout.strip().endswith("OK")
