@@ -84,7 +84,7 @@ def parse():
                     help="rotate mode: replay the timed steps from a CUDA graph or launch them directly")
     ap.add_argument("--replay", default="per_tile", choices=["per_tile", "cluster"],
                     help="value-tiled kernel: ReplayPrep formed per tile, or shared by a head's tiles as one cluster")
-    ap.add_argument("--e2e-copies", default="per_tensor", choices=["per_tensor", "packed"],
+    ap.add_argument("--e2e-copies", default="packed", choices=["packed", "per_tensor"],
                     help="end-to-end leg: copy each input/output tensor, or one packed buffer per step")
     ap.add_argument("--log-format", default="fp32", choices=["fp32", "compact"],
                     help="log entry layout: fp32 [a|b|Lambda], or compact (bf16 a, bf16 b without the delta rule)")
