@@ -9,8 +9,8 @@ import oracle
 from recurrent_state_serving_b200 import synth
 from recurrent_state_serving_b200.runner import DecodeRunner
 
-# Tolerances.  the benchmark spec-level bound: relative L2 error of each step's whole output
-# tensor (and of each checkpointed state) against the fp64 oracle <= 1e-4.  Per
+# Tolerances.  The accuracy bound of this path: relative L2 error of each step's whole
+# output tensor (and of each checkpointed state) against the fp64 oracle <= 1e-4.  Per
 # element we also require |gpu - ref| <= 1e-3 * RMS(ref of that step): the fp32
 # path accumulates d_k-term dot products (error ~ sqrt(d_k) * 2^-24 relative), so a
 # single element 10x above the average allowed error already indicates a bug.
