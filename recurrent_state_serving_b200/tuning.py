@@ -81,6 +81,35 @@ def select_log_cap(measured: dict, higher_is_better: bool = True) -> int:
     return min(pts, key=lambda p: (sign * p[1], p[0]))[0]
 
 
+def select_from_bench_lines(lines) -> dict:
+    """Best interval per operator configuration from bench JSON lines.
+
+    Each line is one ``bench.py --log-cap L`` run (a JSON object, or its text).  Lines
+    are grouped by everything in their ``config`` that does not depend on L (workload
+    shape, decay, update rule, log layout, batch, GPU count); reference-arm lines and
+    lines without a value are skipped.  Returns {group key: (best L, {L: value})}, the
+    key being the workload name without its ``_L<n>`` part plus the log layout."""
+    import json
+    import re
+
+    groups: dict = {}
+    for ln in lines:
+        d = json.loads(ln) if isinstance(ln, str) else ln
+        if not isinstance(d, dict) or d.get("impl") == "reference" or d.get("value") is None:
+            continue
+        cfg = d.get("config", {})
+        if "log_cap" not in cfg or "workload" not in cfg:
+            continue
+        L = int(cfg["log_cap"])
+        base = re.sub(r"_L\d+", "", cfg["workload"])
+        key = (base, cfg.get("log_format", "fp32"), int(d.get("n_gpus", 1)))
+        better = d.get("higher_is_better", True)
+        g = groups.setdefault(key, ({}, better))
+        g[0][L] = float(d["value"])
+    return {f"{b} [{fmt}, {n} GPU]": (select_log_cap(vals, better), vals)
+            for (b, fmt, n), (vals, better) in groups.items()}
+
+
 def sweep_table(wl: Workload, candidates=DEFAULT_CANDIDATES, log_format: str = "fp32"):
     """(L, bytes per head-step, bytes relative to the eager step) for each candidate."""
     eager = traffic.eager_head_step(wl)
@@ -98,7 +127,16 @@ def main(argv=None):
     ap.add_argument("--workload", default="gla_rwkv6_diag", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--log-format", default="fp32", choices=["fp32", "compact"])
     ap.add_argument("--candidates", default=",".join(str(c) for c in DEFAULT_CANDIDATES))
+    ap.add_argument("--from-bench", default=None,
+                    help="file of bench.py JSON lines (one per --log-cap run): print the measured pick")
     a = ap.parse_args(argv)
+    if a.from_bench:
+        with open(a.from_bench) as f:
+            lines = [ln for ln in f if ln.strip().startswith("{")]
+        for key, (best, vals) in sorted(select_from_bench_lines(lines).items()):
+            rates = ", ".join(f"L={L}: {v:.4g}" for L, v in sorted(vals.items()))
+            print(f"{key}: measured best L = {best} ({rates})")
+        return
     wl = synth.WORKLOADS[a.workload]
     cands = [int(x) for x in a.candidates.split(",") if x]
     for L, b, r in sweep_table(wl, cands, a.log_format):

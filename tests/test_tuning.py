@@ -122,3 +122,35 @@ def test_server_takes_the_modelled_interval():
     s = DecodeServer(log_cap="auto", log_format="compact", **kw)
     assert s.log_cap == 16 and s.pool.log_cap == 16 and s.pool.log.shape[3] == 16
     assert DecodeServer(log_cap=5, **kw).log_cap == 5
+
+
+def test_pick_from_bench_lines(tmp_path, capsys):
+    """bench.py lines of an interval sweep (as --log-cap L runs print them) give the
+    measured best interval per workload and log layout; reference lines are ignored."""
+    import json
+
+    import bench
+    lines = []
+    for L, v in {4: 52.9e6, 8: 57.7e6, 16: 54.1e6, 32: 51.0e6}.items():
+        wl = synth.GLA_DIAG.with_(log_cap=L)
+        lines.append(json.dumps({"value": v, "higher_is_better": True, "n_gpus": 1,
+                                 "config": bench.config_of(wl, 1)}))
+    for L, v in {8: 72.77e6, 16: 75.86e6, 32: 71.76e6}.items():
+        wl = synth.RETNET.with_(log_cap=L)
+        lines.append(json.dumps({"value": v, "higher_is_better": True, "n_gpus": 1,
+                                 "config": bench.config_of(wl, 1, log_format="compact")}))
+    ref = synth.GLA_DIAG.with_(log_cap=4)
+    lines.append(json.dumps({"impl": "reference", "value": 1e12, "n_gpus": 1,
+                             "config": bench.config_of(ref, 1)}))
+    picks = tuning.select_from_bench_lines(lines)
+    assert len(picks) == 2
+    gla = next(v for k, v in picks.items() if k.startswith("gla_rwkv6_diag_b64_h16_d128 [fp32"))
+    ret = next(v for k, v in picks.items() if "retnet" in k and "[compact" in k)
+    assert gla[0] == 8 and sorted(gla[1]) == [4, 8, 16, 32]
+    assert ret[0] == 16
+    # the same through the command line, from a file with other output mixed in
+    f = tmp_path / "sweep.jsonl"
+    f.write_text("some log line\n" + "\n".join(lines) + "\n")
+    tuning.main(["--from-bench", str(f)])
+    out = capsys.readouterr().out
+    assert "measured best L = 8" in out and "measured best L = 16" in out
