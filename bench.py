@@ -2,12 +2,26 @@
 """Benchmark of the base + log recurrent-state decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--log-cap L] [--batch B]
+                    [--workload NAME] [--log-cap L] [--batch B] [--subs LIST] [--merge-legs LIST]
 
 A step is one decode step of the whole batch over all layers of the workload (one
 library call per layer), with every slot advancing by one token; merges happen on
 each slot's own merge step inside the same call.  Inputs are seeded synthetic
 tensors resident in HBM before timing starts.
+
+The headline workload is the largest one: KDA-style per-key decay with the delta
+rule, 24 layers x batch 256 x 32 heads, d = 128, log capacity L = 16 (12 GiB of
+base state).  Slot phases are spread (``--phases spread``, default): slot b of slot
+group g starts its merge cycle at offset (o_b + g * batch) mod L, o_b = b (or the
+workload's own random stagger, RetNet), so every launch of a batch of at least L
+slots carries exactly its 1/L share of merge steps and any window of timed steps is
+the amortised step.  The JSON line records the live-entry histogram of the timed
+launches.  ``--phases workload`` keeps the workload's own offsets for every group.
+
+Besides the headline, the line carries sub-records (``--subs``), each with its own
+steps/s, roofline and eager comparison, and merge legs (``--merge-legs``) that time
+standalone ``dl_merge`` of full logs and ``dl_materialize``.  A sub-record's step
+count is at least K, raised so its timed region is a few ms, and a multiple of L.
 
 Cold L2 between steps, two ways (``--l2``):
   rotate (default)  inputs larger than L2: the pool holds R disjoint copies of the
@@ -35,6 +49,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -49,8 +64,16 @@ METRIC = "decode head-steps/s (batch x heads x layers)"
 UNIT = "head-steps/s"
 FLUSH_BYTES = 256 << 20
 ROTATE_MIN_BYTES = 384 << 20  # base-state bytes of one rotation: three times L2 (126 MB)
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "step_kernel_traffic.txt")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 CSRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc")
+DEFAULT_WORKLOAD = "kda_diag_delta"
+DEFAULT_SUBS = "gla_rwkv6_diag:b64:L8,retnet_scalar:b64,retnet_scalar:b256,retnet_scalar:b1024,gdn_gva:b1"
+DEFAULT_MERGE_LEGS = "kda_diag_delta,retnet_scalar:b256"
+SUB_MIN_MS = 3.0            # a sub-record's timed region is at least about this long
+SUB_MAX_STEPS = 4096
+HOST_INPUT_BYTES = 128 << 20  # distinct seeded steps generated per workload (host side)
+DELTA_READING = ("decayed state: b_t = beta_t (v_t - (Diag(exp lambda_t) S_{t-1})^T k_t), "
+                 "the gated delta rule of GDN/KDA (DL_UPDATE_DELTA)")
 
 
 def kernel_source_hash() -> str:
@@ -62,20 +85,28 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="gla_rwkv6_diag")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--log-cap", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--subs", default=DEFAULT_SUBS,
+                    help="comma list of name[:bB][:LL] sub-records, or 'none'")
+    ap.add_argument("--merge-legs", default=DEFAULT_MERGE_LEGS,
+                    help="comma list of name[:bB][:LL] workloads whose dl_merge/dl_materialize are timed, or 'none'")
+    ap.add_argument("--phases", default="spread", choices=["spread", "workload"],
+                    help="slot merge phases: spread over each launch, or the workload's own offsets")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--traffic-from", default=None,
-                    help="write profiles/step_kernel_traffic.txt from an ncu csv and exit")
+                    help="append a record to profiles/dram_traffic.txt from an ncu csv and exit")
+    ap.add_argument("--traffic-kind", default="decode", choices=["decode", "eager", "merge", "materialize"],
+                    help="which launches an ncu csv given with --traffic-from holds")
     ap.add_argument("--tile-v", type=int, default=0,
                     help="work-unit width: 0 automatic, 16/32 value tiles, 128 whole heads")
     ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
@@ -88,12 +119,34 @@ def parse():
                     help="end-to-end leg: copy each input/output tensor, or one packed buffer per step")
     ap.add_argument("--log-format", default="fp32", choices=["fp32", "compact"],
                     help="log entry layout: fp32 [a|b|Lambda], or compact (bf16 a, bf16 b without the delta rule)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def parse_spec(spec: str):
+    """'name[:bB][:LL]' -> a synth workload with that batch / log capacity."""
+    from recurrent_state_serving_b200 import synth
+    parts = spec.strip().split(":")
+    if parts[0] not in synth.WORKLOADS:
+        raise SystemExit(f"unknown workload {parts[0]!r} (known: {', '.join(sorted(synth.WORKLOADS))})")
+    wl = synth.WORKLOADS[parts[0]]
+    for p in parts[1:]:
+        if p.startswith("b"):
+            wl = wl.with_(batch=int(p[1:]))
+        elif p.startswith("L"):
+            wl = wl.with_(log_cap=int(p[1:]))
+        else:
+            raise SystemExit(f"bad workload spec {spec!r}")
+    return wl
+
+
+def spec_list(text: str):
+    if not text or text.strip().lower() == "none":
+        return []
+    return [parse_spec(s) for s in text.split(",") if s.strip()]
 
 
 def workload(a):
-    from recurrent_state_serving_b200 import synth
-    wl = synth.WORKLOADS[a.workload]
+    wl = parse_spec(a.workload)
     if a.log_cap:
         wl = wl.with_(log_cap=a.log_cap)
     if a.batch:
@@ -110,6 +163,71 @@ def rotation_groups(wl, l2_mode: str) -> int:
     return max(1, -(-ROTATE_MIN_BYTES // step_state))
 
 
+def phase_offsets(wl, n_groups: int, mode: str = "spread") -> np.ndarray:
+    """Staggering offsets [n_groups, batch]: how many untimed steps each slot of each
+    group takes before the common steps.
+
+    spread    slot b of group g: (o_b + g * batch) mod L with o_b = b, or the
+              workload's own random offset when it is staggered.  A batch of at least
+              L slots (and o_b = b) then holds every live length 0..L-1 equally in
+              every launch; smaller batches continue the phase sequence across groups.
+    workload  the workload's own offsets (zeros unless staggered) for every group."""
+    from recurrent_state_serving_b200 import synth
+    own = synth.slot_offsets(wl)
+    if mode == "workload":
+        return np.tile(own, (n_groups, 1))
+    if mode != "spread":
+        raise ValueError(mode)
+    base = own if wl.staggered else np.arange(wl.batch)
+    g = np.arange(n_groups)[:, None]
+    return ((base[None, :] + g * wl.batch) % wl.log_cap).astype(np.int64)
+
+
+def live_entries(offsets, step_index: int, n_groups: int, log_cap: int):
+    """Live log entries each slot of the group stepped at global step ``step_index``
+    holds when the step starts: that group has taken step_index // n_groups steps
+    before it, after its staggering pre-steps (the same offsets for every group)."""
+    return (offsets + step_index // n_groups) % log_cap
+
+
+def group_live_entries(group_offsets, step_index: int, log_cap: int):
+    """live_entries() with each group's own offsets ([n_groups, batch])."""
+    R = group_offsets.shape[0]
+    return (group_offsets[step_index % R] + step_index // R) % log_cap
+
+
+def timed_window_bytes(wl, group_offsets, first: int, K: int, log_format: str = "fp32"):
+    """Algorithmic bytes of global steps first .. first+K-1 (all layers and heads)
+    and the histogram of the slots' live entries at those steps."""
+    from recurrent_state_serving_b200 import traffic
+    L = wl.log_cap
+    per_c = [traffic.deferred_head_step(wl, c, merge=(c == L - 1), log_format=log_format) for c in range(L)]
+    hist = np.zeros(L, np.int64)
+    for j in range(first, first + K):
+        hist += np.bincount(group_live_entries(group_offsets, j, L), minlength=L)
+    per_slot = float(np.dot(hist, per_c))
+    scale = wl.n_heads * wl.n_layers
+    return per_slot * scale, hist
+
+
+def sub_steps(wl, K: int, log_format: str = "fp32") -> int:
+    """Timed steps of a sub-record: at least K, enough for about SUB_MIN_MS at 5 TB/s
+    (plus 3 us per launch), a multiple of L, at most SUB_MAX_STEPS."""
+    from recurrent_state_serving_b200 import traffic
+    est_ms = (traffic.deferred_cycle_average(wl, log_format) * wl.units_per_step / 5e12 * 1e3
+              + 3e-3 * wl.n_layers)
+    n = max(K, int(math.ceil(SUB_MIN_MS / est_ms)))
+    n = -(-n // wl.log_cap) * wl.log_cap
+    return min(n, max(K, SUB_MAX_STEPS))
+
+
+def distinct_steps(wl) -> int:
+    """Distinct seeded input steps generated for a workload (cycled while timing)."""
+    from recurrent_state_serving_b200 import traffic
+    per = traffic.token_bytes(wl) * wl.units_per_step
+    return int(max(2, min(wl.steps, 256 // wl.n_layers, HOST_INPUT_BYTES // max(1.0, per))))
+
+
 def l2_description(wl, l2_mode: str, launch: str) -> str:
     if l2_mode == "flush":
         return ("flushed before every timed step, outside the timed interval: 256 MiB write, then "
@@ -121,23 +239,42 @@ def l2_description(wl, l2_mode: str, launch: str) -> str:
             f"{'replayed from one CUDA graph' if launch == 'graph' else 'launched directly'}")
 
 
-def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph", log_format="fp32", replay="per_tile"):
+def phases_description(wl, mode: str) -> str:
+    if mode == "workload":
+        return ("each group keeps the workload's own offsets: "
+                + ("random in [0, L) per slot" if wl.staggered else "all slots merge on the same step"))
+    src = "the workload's random offset o_b in [0, L)" if wl.staggered else "o_b = b"
+    return (f"spread: slot b of group g starts its merge cycle at (o_b + g*batch) mod L, {src}; "
+            f"every launch of >= L slots holds each live length 0..L-1 equally")
+
+
+def config_of(wl, n_gpus, tile_v=0, l2_mode="rotate", launch="graph", log_format="fp32", replay="per_tile",
+              phases="spread"):
     suffix = "" if log_format == "fp32" else f"_{log_format}log"
-    return {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}{suffix}",
-            "tile_v": tile_v or "auto", "log_format": log_format, "replay": replay,
-            "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
-            "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
-            "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
-            "l2": l2_description(wl, l2_mode, launch),
-            "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
+    cfg = {"workload": f"{wl.name}_b{wl.batch}_h{wl.n_heads}_d{wl.d_k}_L{wl.log_cap}{suffix}",
+           "tile_v": tile_v or "auto", "log_format": log_format, "replay": replay,
+           "layers": wl.n_layers, "batch_per_gpu": wl.batch, "heads": wl.n_heads,
+           "kheads": wl.n_kheads, "d_k": wl.d_k, "d_v": wl.d_v, "log_cap": wl.log_cap,
+           "decay": wl.decay, "update": wl.update, "inputs": wl.in_dtype, "state": "fp32",
+           "phases": phases_description(wl, phases),
+           "l2": l2_description(wl, l2_mode, launch),
+           "parallelism": f"replicas x{n_gpus} (independent slots, no collective)"}
+    if wl.update == "delta":
+        cfg["delta_reading"] = DELTA_READING
+    return cfg
 
 
-def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str) -> str:
-    """Text for profiles/step_kernel_traffic.txt from an ncu --csv export of
-    dram__bytes_read.sum and dram__bytes_write.sum over consecutive launches of the
-    hot kernel (a whole merge cycle of every slot group: rotation groups x log
-    capacity launches, so the mix of append and merge launches matches the timed
-    region).  Run: python bench.py --traffic-from <csv>."""
+def workload_key(wl, log_format="fp32") -> str:
+    return config_of(wl, 1, log_format=log_format)["workload"]
+
+
+def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str, kind: str = "decode") -> str:
+    """One record for profiles/dram_traffic.txt from an ncu --csv export of
+    dram__bytes_read.sum and dram__bytes_write.sum (and, when present, the L2 write
+    sectors lts__t_sectors_srcunit_tex_op_write.sum) over consecutive launches of
+    one kernel.  For decode launches the capture should span a whole cycle of
+    launch mixes, so append and merge heads mix as in the timed region.
+    Run: python bench.py --traffic-from <csv> --traffic-kind KIND [--workload ...]."""
     import csv
     import re
     rows = list(csv.reader(open(csv_path)))
@@ -145,27 +282,64 @@ def traffic_summary_from_ncu(csv_path: str, workload_key: str, kernel_regex: str
     hdr = rows[i]
     kn, mn, mv = hdr.index("Kernel Name"), hdr.index("Metric Name"), hdr.index("Metric Value")
     mu = hdr.index("Metric Unit") if "Metric Unit" in hdr else None
-    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
-    per = {}
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9,
+             "sector": 1, "Ksector": 1e3, "Msector": 1e6, "Gsector": 1e9}
+    per, l2w = {}, {}
     idcol = hdr.index("ID") if "ID" in hdr else None
     for r in rows[i + 1:]:
         if len(r) <= mv or not re.search(kernel_regex, r[kn]):
             continue
-        if r[mn] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
-            continue
-        v = float(r[mv].replace(",", "")) * scale.get(r[mu] if mu is not None else "byte", 1)
         key = r[idcol] if idcol is not None else len(per)
-        per[key] = per.get(key, 0.0) + v
+        v = float(r[mv].replace(",", "")) * scale.get(r[mu] if mu is not None else "byte", 1)
+        if r[mn] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            per[key] = per.get(key, 0.0) + v
+        elif r[mn] == "lts__t_sectors_srcunit_tex_op_write.sum":
+            l2w[key] = l2w.get(key, 0.0) + 32.0 * v
     vals = list(per.values())
     if not vals:
         raise SystemExit("no matching launches in " + csv_path)
     avg = sum(vals) / len(vals)
-    return (f"# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the hot kernel,\n"
-            f"# averaged over {len(vals)} consecutive launches (a whole merge cycle of every\n"
-            f"# slot group, so append and merge launches mix as in the timed region).\n"
-            f"workload = {workload_key}\nkernel_sha = {kernel_source_hash()}\n"
+    text = (f"workload = {workload_key}\nkind = {kind}\nkernel_sha = {kernel_source_hash()}\n"
             f"launches = {len(vals)}\ndram_bytes_per_launch = {avg:.0f}\n"
             f"min_launch_bytes = {min(vals):.0f}\nmax_launch_bytes = {max(vals):.0f}\n")
+    if l2w:
+        text += f"l2_write_bytes_per_launch = {sum(l2w.values()) / len(l2w):.0f}\n"
+    return text
+
+
+def traffic_records(path=None):
+    """Records of profiles/dram_traffic.txt: each starts at a 'workload = ' line."""
+    path = path or PROFILE_TRAFFIC
+    if not os.path.exists(path):
+        return []
+    recs, cur = [], None
+    for line in open(path):
+        if "=" not in line or line.lstrip().startswith("#"):
+            continue
+        k, v = (x.strip() for x in line.split("=", 1))
+        if k == "workload":
+            cur = {}
+            recs.append(cur)
+        if cur is not None:
+            cur[k] = v
+    return recs
+
+
+def recorded_traffic(workload_key, kind="decode", field="dram_bytes_per_launch"):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
+    when there is none for this workload and kind, or the kernel source changed
+    since it was taken."""
+    sha = kernel_source_hash()
+    for r in traffic_records():
+        if r.get("workload") != workload_key or r.get("kind", "decode") != kind:
+            continue
+        if r.get("kernel_sha") != sha:
+            continue
+        try:
+            return float(r[field])
+        except (KeyError, ValueError):
+            return None
+    return None
 
 
 def measured_peaks():
@@ -174,24 +348,6 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
     return 6650.0, "fallback (6.65 TB/s)"
-
-
-def recorded_traffic(workload_key):
-    """Per-launch DRAM bytes of the step kernel from a committed ncu summary, or None
-    when the summary is missing or the kernel source changed since it was taken."""
-    if not os.path.exists(PROFILE_TRAFFIC):
-        return None
-    kv = {}
-    for line in open(PROFILE_TRAFFIC):
-        if "=" in line and not line.lstrip().startswith("#"):
-            k, v = line.split("=", 1)
-            kv[k.strip()] = v.strip()
-    if kv.get("kernel_sha") != kernel_source_hash() or kv.get("workload") != workload_key:
-        return None
-    try:
-        return float(kv["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
 
 
 # ---------------------------------------------------------------------------------
@@ -281,13 +437,6 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms / 1e3)
 
 
-def live_entries(offsets, step_index: int, n_groups: int, log_cap: int):
-    """Live log entries each slot of the group stepped at global step ``step_index``
-    holds when the step starts: that group has taken step_index // n_groups steps
-    before it, after its staggering pre-steps."""
-    return (offsets + step_index // n_groups) % log_cap
-
-
 def graph_upload(graph, stream) -> bool:
     """Upload an instantiated CUDA graph to the device ahead of its first replay, so
     the replay inside the timed interval carries no upload work."""
@@ -354,53 +503,52 @@ def packed_views(buf, spec, offs):
     return out
 
 
-def run_gpu(a, wl, rank, world, dist):
-    import torch
-    from recurrent_state_serving_b200 import deltalog as dl
-    from recurrent_state_serving_b200 import synth, traffic
-    from recurrent_state_serving_b200.runner import DecodeRunner
+class GpuContext:
+    """Device, ranks, clocks and the timing loop shared by every leg."""
 
-    dev = torch.device("cuda", torch.cuda.current_device())
-    if a.l2 == "flush":
-        flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-        flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-        flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    def __init__(self, a, world, dist):
+        import torch
+        self.torch = torch
+        self.a, self.world, self.dist = a, world, dist
+        self.dev = torch.device("cuda", torch.cuda.current_device())
+        self.sampler = ClockSampler(self.dev.index)
+        self.sampler.start()
+        self.launches = 0
+        if a.l2 == "flush":
+            self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+            self.flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+            self.flush_sink = torch.empty((), dtype=torch.float32, device=self.dev)
+        self.graph_uploaded = None
 
-    def flush_l2():
-        flush.zero_()
-        torch.sum(flush_rd, dim=0, out=flush_sink)
-    L, K, W = wl.log_cap, a.steps, a.warmup
-    ndist = max(1, min(wl.steps, 256 // wl.n_layers))
+    def flush_l2(self):
+        self.flush.zero_()
+        self.torch.sum(self.flush_rd, dim=0, out=self.flush_sink)
 
-    def barrier_sync():
-        torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
+    def barrier_sync(self):
+        self.torch.cuda.synchronize()
+        if self.dist is not None:
+            self.dist.barrier()
+        self.torch.cuda.synchronize()
 
-    def reduce_max(x):
-        return max_over_ranks(x, dist, dev)
+    def reduce_max(self, x):
+        return max_over_ranks(x, self.dist, self.dev)
 
-    host_inputs = [[synth.step_inputs(wl, t, l) for l in range(wl.n_layers)] for t in range(ndist)]
-    sampler = ClockSampler(dev.index)
-    sampler.start()
-
-    R = rotation_groups(wl, a.l2)
-    use_graph = a.l2 == "rotate" and a.launch == "graph"
-    graph_info = {}
-
-    def timed(calls_for_step, n_steps, graph_ok=True):
-        """calls_for_step(j) -> callables issued for global step j (one per layer).
-        Returns the timed interval in ms (sum of the per-step intervals when flushing)."""
+    def timed(self, calls_for_step, n_steps, W, graph_ok=True, per_step_events=False):
+        """calls_for_step(j) -> callables issued for global step j.  Steps 0..W-1 run
+        untimed, W..W+n_steps-1 timed.  Returns the timed interval in ms (the sum of
+        per-step intervals when flushing or with per_step_events)."""
+        torch = self.torch
+        a = self.a
         for j in range(W):
             for c in calls_for_step(j):
                 c()
-        barrier_sync()
-        if a.l2 == "flush":
+        self.barrier_sync()
+        if a.l2 == "flush" or per_step_events:
             t0 = time.time()
             evs = []
             for i in range(n_steps):
-                flush_l2()
+                if a.l2 == "flush":
+                    self.flush_l2()
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
@@ -408,11 +556,11 @@ def run_gpu(a, wl, rank, world, dist):
                     c()
                 e1.record()
                 evs.append((e0, e1))
-            barrier_sync()
-            sampler.mark(t0, time.time())
+            self.barrier_sync()
+            self.sampler.mark(t0, time.time())
             return sum(e0.elapsed_time(e1) for e0, e1 in evs)
         g = None
-        if use_graph and graph_ok:
+        if a.launch == "graph" and graph_ok:
             g = torch.cuda.CUDAGraph()
             cs = torch.cuda.Stream()
             cs.wait_stream(torch.cuda.current_stream())
@@ -423,8 +571,9 @@ def run_gpu(a, wl, rank, world, dist):
                         c()
                 g.capture_end()
             torch.cuda.current_stream().wait_stream(cs)
-            graph_info["uploaded"] = graph_upload(g, torch.cuda.current_stream())
-            barrier_sync()
+            up = graph_upload(g, torch.cuda.current_stream())
+            self.graph_uploaded = up if self.graph_uploaded is None else (self.graph_uploaded and up)
+            self.barrier_sync()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         t0 = time.time()
@@ -436,216 +585,375 @@ def run_gpu(a, wl, rank, world, dist):
                 for c in calls_for_step(W + i):
                     c()
         e1.record()
-        barrier_sync()
-        sampler.mark(t0, time.time())
+        self.barrier_sync()
+        self.sampler.mark(t0, time.time())
         ms = e0.elapsed_time(e1)
         del g
         return ms
 
-    # ---- deferred (the product path) ----
-    r = DecodeRunner(wl, device=str(dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format,
-                     replay=a.replay)
-    r.load_initial_state()
-    r.run_presteps()
-    dev_inputs = [[r.device_inputs(x) for x in per_layer] for per_layer in host_inputs]
-    outs = [torch.empty(wl.batch, wl.n_heads, wl.d_v, dtype=torch.float32, device=dev)
-            for _ in range(wl.n_layers)]
 
-    def check(st):
-        if st != 0:
-            raise dl.DeltaLogError(st, "dl_decode_step")
+def check_status(st, what="dl_decode_step"):
+    if st != 0:
+        from recurrent_state_serving_b200 import deltalog as dl
+        raise dl.DeltaLogError(st, what)
 
-    def prepared_calls(kind, runner, cache):
-        """Step j: group j mod R, step inputs j mod ndist (argument blocks built once)."""
-        def calls(j):
-            key = (j % R, j % ndist)
-            if key not in cache:
-                g, t = key
-                cache[key] = [dl.PreparedStep(kind, runner.pool, l, runner.group_slots[g], x["q"], x["k"],
-                                              x["v"], x["lam"], x["beta"], outs[l], wl.lambda_const)
-                              for l, x in enumerate(dev_inputs[t])]
-            return [(lambda p=p: check(p())) for p in cache[key]]
-        return calls
 
-    total_ms = timed(prepared_calls("decode", r, {}), K)
-    assert r.errors() == 0, "device error bits set during the benchmark"
-    max_ms = reduce_max(total_ms)
-    value = whole_job_rate(wl.units_per_step * K, world, max_ms)
+class WorkloadSetup:
+    """A workload's distinct seeded inputs on the device and its output buffers."""
 
-    # algorithmic bytes of the timed launches: each slot enters its step with the
-    # live entries of its own auto-merge cycle of length L
-    offs = synth.slot_offsets(wl)
-    bytes_total = 0.0
-    for i in range(K):
-        c = live_entries(offs, W + i, R, L)
-        per_slot = [traffic.deferred_head_step(wl, int(cb), merge=(cb == L - 1), log_format=a.log_format)
-                    for cb in c]
-        bytes_total += sum(per_slot) * wl.n_heads * wl.n_layers
-    launches = K * wl.n_layers
-    achieved_gbs = bytes_total / (total_ms / 1e3) / 1e9
+    def __init__(self, ctx, wl):
+        from recurrent_state_serving_b200 import synth
+        from recurrent_state_serving_b200.runner import _to_dev_input
+        torch = ctx.torch
+        self.wl = wl
+        self.ndist = distinct_steps(wl)
+        self.host = [[synth.step_inputs(wl, t, l) for l in range(wl.n_layers)] for t in range(self.ndist)]
+        self.dev = [[{k: _to_dev_input(v, wl.in_dtype if k in ("q", "k", "v") else "f32", ctx.dev)
+                      for k, v in x.items()} for x in per_layer] for per_layer in self.host]
+        self.outs = [torch.empty(wl.batch, wl.n_heads, wl.d_v, dtype=torch.float32, device=ctx.dev)
+                     for _ in range(wl.n_layers)]
+
+    def prestep_inputs(self, p, layer):
+        return self.dev[p % self.ndist][layer]
+
+
+def prepared_calls(kind, wl, runner, setup, R, cache):
+    """Step j: group j mod R, distinct inputs j mod ndist (argument blocks built once)."""
+    from recurrent_state_serving_b200 import deltalog as dl
+
+    def calls(j):
+        key = (j % R, j % setup.ndist)
+        if key not in cache:
+            g, t = key
+            cache[key] = [dl.PreparedStep(kind, runner.pool, l, runner.group_slots[g], x["q"], x["k"],
+                                          x["v"], x["lam"], x["beta"], setup.outs[l], wl.lambda_const)
+                          for l, x in enumerate(setup.dev[t])]
+        return [(lambda p=p: check_status(p())) for p in cache[key]]
+    return calls
+
+
+def roofline_record(achieved_gbs, kernel, launches, total_ms, bytes_per_launch, traffic_bytes):
     peak, peak_src = measured_peaks()
-    key = config_of(wl, world, log_format=a.log_format)["workload"]
-    dram = recorded_traffic(key)
-    roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
+    return {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved_gbs / peak, 4), "peak_source": peak_src,
-            "traffic": dram, "algorithmic_bytes_per_launch": round(bytes_total / launches),
-            "kernel": res_kernel_name(wl, a.tile_v), "launches_timed": launches,
+            "traffic": traffic_bytes, "algorithmic_bytes_per_launch": round(bytes_per_launch),
+            "kernel": kernel, "launches_timed": launches,
             "avg_launch_us": round(total_ms * 1e3 / launches, 3),
             "frac_of_8tbs_spec": round(achieved_gbs / 8000.0, 4)}
 
-    result = {"value": value, "ms_per_step": max_ms / K, "roofline": roof, "gpu_launches": launches,
-              "rotation_groups": R}
-    if use_graph:
-        result["graph_uploaded"] = graph_info.get("uploaded")
 
-    # ---- eager comparison (same workload, full read-modify-write each step) ----
-    if not a.no_eager:
-        re_ = DecodeRunner(wl, device=str(dev), mode="eager", tile_v=a.tile_v, n_groups=R)
-        re_.load_initial_state()
-        ms_e = timed(prepared_calls("eager", re_, {}), K)
-        assert re_.errors() == 0
-        tot_e = reduce_max(ms_e)
+def measure_decode(ctx, wl, K, W, *, eager=True, keep=False):
+    """Deferred decode steps of a workload (the product path), then the in-library
+    eager step on the same workload.  Returns (record, runner and setup when keep)."""
+    from recurrent_state_serving_b200 import traffic
+    from recurrent_state_serving_b200.runner import DecodeRunner
+    torch = ctx.torch
+    a = ctx.a
+    setup = WorkloadSetup(ctx, wl)
+    R = rotation_groups(wl, a.l2)
+    goffs = phase_offsets(wl, R, a.phases)
+    r = DecodeRunner(wl, device=str(ctx.dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format,
+                     replay=a.replay, offsets=goffs)
+    r.load_initial_state(on_device=True)
+    r.run_presteps(inputs=setup.prestep_inputs)
+    total_ms = ctx.timed(prepared_calls("decode", wl, r, setup, R, {}), K, W)
+    if r.errors() != 0:
+        raise RuntimeError("device error bits set during the benchmark")
+    max_ms = ctx.reduce_max(total_ms)
+    launches = K * wl.n_layers
+    ctx.launches += launches
+    bytes_total, hist = timed_window_bytes(wl, goffs, W, K, a.log_format)
+    achieved = bytes_total / (total_ms / 1e3) / 1e9
+    key = workload_key(wl, a.log_format)
+    units = hist.sum() * wl.n_heads * wl.n_layers
+    rec = {"workload": key, "value": whole_job_rate(wl.units_per_step * K, ctx.world, max_ms), "unit": UNIT,
+           "ms_per_step": max_ms / K, "steps": K, "warmup": W, "rotation_groups": R,
+           "roofline": roofline_record(achieved, res_kernel_name(wl, a.tile_v), launches, total_ms,
+                                       bytes_total / launches, recorded_traffic(key, "decode")),
+           "live_entries": {"hist": [int(x) for x in hist],
+                            "merge_share": round(float(hist[-1]) / max(1, hist.sum()), 4),
+                            "bytes_per_head_step": round(bytes_total / units, 1),
+                            "cycle_average_model": round(traffic.deferred_cycle_average(wl, a.log_format), 1)},
+           "deferred_bytes_per_step": round(bytes_total / K)}
+    if wl.update == "delta":
+        rec["delta_reading"] = DELTA_READING
+    if eager and not a.no_eager:
+        re_ = DecodeRunner(wl, device=str(ctx.dev), mode="eager", tile_v=a.tile_v, n_groups=R)
+        re_.load_initial_state(on_device=True)
+        ms_e = ctx.timed(prepared_calls("eager", wl, re_, setup, R, {}), K, W)
+        if re_.errors() != 0:
+            raise RuntimeError("device error bits set in the eager leg")
+        ctx.launches += launches
+        tot_e = ctx.reduce_max(ms_e)
         eb = traffic.eager_head_step(wl) * wl.units_per_step * K
-        result["eager"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_e),
-                           "ms_per_step": tot_e / K,
-                           "algorithmic_bytes_per_step": round(eb / K),
-                           "achieved_gbs": round(eb / (ms_e / 1e3) / 1e9, 1)}
-        result["deferred_bytes_per_step"] = round(bytes_total / K)
+        ach_e = eb / (ms_e / 1e3) / 1e9
+        rec["eager"] = {"value": whole_job_rate(wl.units_per_step * K, ctx.world, tot_e),
+                        "ms_per_step": tot_e / K, "algorithmic_bytes_per_step": round(eb / K),
+                        "achieved_gbs": round(ach_e, 1), "frac": round(ach_e / measured_peaks()[0], 4),
+                        "kernel": "dl::step_kernel (eager flag)",
+                        "traffic": recorded_traffic(key, "eager")}
+        rec["deferred_over_eager"] = round(rec["value"] / rec["eager"]["value"], 3)
+        rec["eager_bytes_over_deferred"] = round(eb / bytes_total, 3)
         del re_
-        torch.cuda.empty_cache()
+    if keep:
+        return rec, (r, setup, R, goffs)
+    del r, setup
+    torch.cuda.empty_cache()
+    return rec, None
 
-    # ---- end to end through the public API with host buffers ----
-    if not a.no_e2e:
-        # Inputs and outputs are double-buffered (set j % 2 for step j); the serial
-        # form uses set 0 only.  --e2e-copies packed lays each step's inputs (all
-        # layers) out in one pinned host buffer and every layer's output in one device
-        # buffer, so a step is one upload and one download; per_tensor copies each
-        # input and output tensor on its own.
-        if a.e2e_copies == "packed":
-            spec = [{k: (None if v is None else (tuple(v.shape), v.dtype)) for k, v in x.items()}
-                    for x in dev_inputs[0]]
-            in_bytes, in_offs = pack_layout(spec)
-            host_pk = []
-            for per_layer in dev_inputs:
-                hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
-                for view, x in zip(packed_views(hb, spec, in_offs), per_layer):
-                    for k, v in x.items():
-                        if v is not None:
-                            view[k].copy_(v.cpu())
-                host_pk.append(hb)
-            out_spec = [{"o": (tuple(o.shape), o.dtype)} for o in outs]
-            out_bytes, out_offs = pack_layout(out_spec)
-            h2d, d2h = in_bytes, out_bytes   # the buffers copied (tensors plus alignment padding)
-            stage_buf = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-            stage = [packed_views(sb, spec, in_offs) for sb in stage_buf]
-            out_buf = [torch.empty(out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
-            outs_e = [[v["o"] for v in packed_views(ob, out_spec, out_offs)] for ob in out_buf]
-            out_host = [torch.empty(out_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
 
-            def upload(t, b):
-                stage_buf[b].copy_(host_pk[t], non_blocking=True)
+def measure_merge(ctx, wl, K, W):
+    """Standalone merge (dl_merge of full logs, c = L on every head) and materialise
+    (dl_materialize of the same logs, pool unchanged), all layers per step."""
+    from recurrent_state_serving_b200 import deltalog as dl
+    from recurrent_state_serving_b200 import traffic
+    from recurrent_state_serving_b200.runner import DecodeRunner
+    torch = ctx.torch
+    a = ctx.a
+    setup = WorkloadSetup(ctx, wl)
+    R = rotation_groups(wl, a.l2)
+    r = DecodeRunner(wl, device=str(ctx.dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format,
+                     replay=a.replay, offsets=np.zeros((R, wl.batch), np.int64))
+    r.load_initial_state(on_device=True)
+    L = wl.log_cap
+    appends = {}
 
-            def download(b):
-                out_host[b].copy_(out_buf[b], non_blocking=True)
-        else:
-            pin = lambda t: None if t is None else t.cpu().pin_memory()
-            host_dev = [[{k: pin(v) for k, v in x.items()} for x in per_layer] for per_layer in dev_inputs]
-            h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
-            d2h = sum(o.numel() * o.element_size() for o in outs)
-            stage = [[{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
-                      for x in dev_inputs[0]] for _ in range(2)]
-            outs_e = [[torch.empty_like(o) for o in outs] for _ in range(2)]
-            out_host = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
+    def fill(g):
+        # L appends per layer: every head of the group holds a full log (c = L)
+        for t in range(L):
+            key = (g, t % setup.ndist)
+            if key not in appends:
+                x_l = setup.dev[t % setup.ndist]
+                appends[key] = [dl.PreparedStep("append", r.pool, l, r.group_slots[g], x["q"], x["k"], x["v"],
+                                                x["lam"], x["beta"], None, wl.lambda_const)
+                                for l, x in enumerate(x_l)]
+            for p in appends[key]:
+                check_status(p(), "dl_append")
 
-            def upload(t, b):
-                for l in range(wl.n_layers):
-                    for k, v in host_dev[t][l].items():
-                        if v is not None:
-                            stage[b][l][k].copy_(v, non_blocking=True)
+    dense = torch.empty(wl.batch, wl.n_heads, wl.d_k, wl.d_v, dtype=torch.float32, device=ctx.dev)
+    # materialise first (the pool is not changed): back-to-back steps over full logs
+    for g in range(R):
+        fill(g)
 
-            def download(b):
-                for l in range(wl.n_layers):
-                    out_host[b][l].copy_(outs_e[b][l], non_blocking=True)
-        prep_2 = [[[dl.PreparedStep("decode", r.pool, l, gs, s_["q"], s_["k"], s_["v"], s_["lam"],
-                                    s_["beta"], outs_e[b][l], wl.lambda_const) for l, s_ in enumerate(stage[b])]
-                   for b in range(2)] for gs in r.group_slots]
-        copies = ("one H2D copy of the step's packed pinned inputs" if a.e2e_copies == "packed"
-                  else "H2D copies of the step's pinned inputs")
-        copies_out = "one D2H copy of every layer's o_t" if a.e2e_copies == "packed" else "D2H of o_t"
+    def mat_calls(j):
+        g = j % R
+        return [(lambda l=l: dl.dl_materialize(r.pool, l, r.group_slots[g], dense)) for l in range(wl.n_layers)]
+    ms_m = ctx.timed(mat_calls, K, W, graph_ok=False)
+    # merge: each timed step folds one group's full logs; refills are untimed
+    ms_g = 0.0
+    for i in range(W + K):
+        g = i % R
+        if i >= R:
+            fill(g)
+        torch.cuda.synchronize()
+        if a.l2 == "flush":
+            ctx.flush_l2()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        e0.record()
+        for l in range(wl.n_layers):
+            dl.dl_merge(r.pool, l, r.group_slots[g])
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= W:
+            ctx.sampler.mark(t0, time.time())
+            ms_g += e0.elapsed_time(e1)
+    if r.errors() != 0:
+        raise RuntimeError("device error bits set in the merge leg")
+    if int(r.pool.log_len.abs().sum()) != 0 and R == 1:
+        raise RuntimeError("merge left live entries")
+    launches = K * wl.n_layers
+    ctx.launches += 2 * launches
+    per_head = traffic.merge_head(wl, L, a.log_format)
+    tot = per_head * wl.units_per_step * K
+    key = workload_key(wl, a.log_format)
+    out = {}
+    for name, ms in (("merge", ctx.reduce_max(ms_g)), ("materialize", ctx.reduce_max(ms_m))):
+        ach = tot / (ms / 1e3) / 1e9
+        out[name] = {"value": whole_job_rate(wl.units_per_step * K, ctx.world, ms), "unit": "head-merges/s",
+                     "ms_per_step": ms / K, "live_entries": L,
+                     "roofline": roofline_record(ach, "dl::merge_kernel", launches, ms, tot / launches,
+                                                 recorded_traffic(key, name))}
+    del r, setup, dense
+    torch.cuda.empty_cache()
+    return {"workload": key, "bytes_per_head": per_head,
+            "calls": "dl_merge / dl_materialize per layer, every head with c = L live entries", **out}
 
-        def serial_calls(j):
-            t, prep = j % ndist, prep_2[j % R][0]
 
-            def one():
-                upload(t, 0)
-                for p_ in prep:
-                    check(p_())
-                download(0)
-            return [one]
+def measure_e2e(ctx, wl, K, W, runner, setup, R, goffs):
+    """End to end through the public API with host buffers: pinned host inputs ->
+    H2D -> dl_decode_step per layer -> D2H of o_t, all inside the events."""
+    from recurrent_state_serving_b200 import deltalog as dl
+    torch = ctx.torch
+    a = ctx.a
+    dev = ctx.dev
+    r = runner
+    outs = setup.outs
+    if a.e2e_copies == "packed":
+        spec = [{k: (None if v is None else (tuple(v.shape), v.dtype)) for k, v in x.items()}
+                for x in setup.dev[0]]
+        in_bytes, in_offs = pack_layout(spec)
+        host_pk = []
+        for per_layer in setup.dev:
+            hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+            for view, x in zip(packed_views(hb, spec, in_offs), per_layer):
+                for k, v in x.items():
+                    if v is not None:
+                        view[k].copy_(v.cpu())
+            host_pk.append(hb)
+        out_spec = [{"o": (tuple(o.shape), o.dtype)} for o in outs]
+        out_bytes, out_offs = pack_layout(out_spec)
+        h2d, d2h = in_bytes, out_bytes   # the buffers copied (tensors plus alignment padding)
+        stage_buf = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        stage = [packed_views(sb, spec, in_offs) for sb in stage_buf]
+        out_buf = [torch.empty(out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        outs_e = [[v["o"] for v in packed_views(ob, out_spec, out_offs)] for ob in out_buf]
+        out_host = [torch.empty(out_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
 
-        # Pipelined: uploads on one copy stream, the decode calls on the current
-        # stream, downloads on another copy stream, with buffer set j % 2 for step j.
-        # Step j's upload waits until step j-2's kernels have read that set; its
-        # kernels wait for its upload and for step j-2's download of the same
-        # outputs; its download waits for its kernels.  So step j+1's upload and step
-        # j-1's download run while step j computes.
-        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_comp = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
-        last = W + K - 1
+        def upload(t, b):
+            stage_buf[b].copy_(host_pk[t], non_blocking=True)
 
-        def piped_calls(j):
-            t, b = j % ndist, j % 2
-            prep = prep_2[j % R][b]
+        def download(b):
+            out_host[b].copy_(out_buf[b], non_blocking=True)
+    else:
+        pin = lambda t: None if t is None else t.cpu().pin_memory()
+        host_dev = [[{k: pin(v) for k, v in x.items()} for x in per_layer] for per_layer in setup.dev]
+        h2d = sum(v.numel() * v.element_size() for x in host_dev[0] for v in x.values() if v is not None)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        stage = [[{k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
+                  for x in setup.dev[0]] for _ in range(2)]
+        outs_e = [[torch.empty_like(o) for o in outs] for _ in range(2)]
+        out_host = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
 
-            def one():
-                comp = torch.cuda.current_stream()
-                if j == W:
-                    # the timed region starts at the compute stream's start event
-                    s_in.wait_stream(comp)
-                    s_out.wait_stream(comp)
-                s_in.wait_event(ev_comp[b])
-                with torch.cuda.stream(s_in):
-                    upload(t, b)
-                ev_in[b].record(s_in)
-                comp.wait_event(ev_in[b])
-                comp.wait_event(ev_out[b])
-                for p_ in prep:
-                    check(p_())
-                ev_comp[b].record(comp)
-                s_out.wait_event(ev_comp[b])
-                with torch.cuda.stream(s_out):
-                    download(b)
-                ev_out[b].record(s_out)
-                if j == last:
-                    comp.wait_stream(s_out)   # the end event follows the last download
-            return [one]
+        def upload(t, b):
+            for l in range(wl.n_layers):
+                for k, v in host_dev[t][l].items():
+                    if v is not None:
+                        stage[b][l][k].copy_(v, non_blocking=True)
 
-        # the calls a user makes, launched directly (no graph)
-        ms_s = timed(serial_calls, K, graph_ok=False)
-        assert r.errors() == 0
-        tot_s = reduce_max(ms_s)
-        serial = {"value": whole_job_rate(wl.units_per_step * K, world, tot_s), "unit": UNIT,
-                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_s / K,
-                  "copies": a.e2e_copies,
-                  "path": f"one stream: {copies} -> dl_decode_step per layer -> {copies_out}, "
-                          "step after step, all inside the events"}
-        if a.l2 == "rotate":
-            ms_p = timed(piped_calls, K, graph_ok=False)
-            assert r.errors() == 0
-            tot_p = reduce_max(ms_p)
-            result["e2e"] = {"value": whole_job_rate(wl.units_per_step * K, world, tot_p), "unit": UNIT,
-                             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_p / K,
-                             "copies": a.e2e_copies,
-                             "path": f"{copies} (copy stream) -> dl_decode_step per layer (compute "
-                                     f"stream) -> {copies_out} (second copy stream), double-buffered so "
-                                     "that step j+1's upload and step j-1's download overlap step j's "
-                                     "kernels; every copy inside the events"}
-            result["e2e_serial"] = serial
-        else:
-            result["e2e"] = serial
-    result["clocks"] = sampler.stop()
+        def download(b):
+            for l in range(wl.n_layers):
+                out_host[b][l].copy_(outs_e[b][l], non_blocking=True)
+    prep_2 = [[[dl.PreparedStep("decode", r.pool, l, gs, s_["q"], s_["k"], s_["v"], s_["lam"],
+                                s_["beta"], outs_e[b][l], wl.lambda_const) for l, s_ in enumerate(stage[b])]
+               for b in range(2)] for gs in r.group_slots]
+    copies = ("one H2D copy of the step's packed pinned inputs" if a.e2e_copies == "packed"
+              else "H2D copies of the step's pinned inputs")
+    copies_out = "one D2H copy of every layer's o_t" if a.e2e_copies == "packed" else "D2H of o_t"
+    ndist = setup.ndist
+    # the deferred leg ran W + K steps on every group before this leg
+    j0 = W + K
+
+    def serial_calls(j):
+        j = j + j0
+        t, prep = j % ndist, prep_2[j % R][0]
+
+        def one():
+            upload(t, 0)
+            for p_ in prep:
+                check_status(p_())
+            download(0)
+        return [one]
+
+    # Pipelined: uploads on one copy stream, the decode calls on the current
+    # stream, downloads on another copy stream, with buffer set j % 2 for step j.
+    # Step j's upload waits until step j-2's kernels have read that set; its
+    # kernels wait for its upload and for step j-2's download of the same
+    # outputs; its download waits for its kernels.  So step j+1's upload and step
+    # j-1's download run while step j computes.
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    last = W + K - 1
+
+    def piped_calls(jl):
+        j = jl + j0 + W + K
+        t, b = j % ndist, jl % 2
+        prep = prep_2[j % R][b]
+
+        def one():
+            comp = torch.cuda.current_stream()
+            if jl == W:
+                # the timed region starts at the compute stream's start event
+                s_in.wait_stream(comp)
+                s_out.wait_stream(comp)
+            s_in.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_in):
+                upload(t, b)
+            ev_in[b].record(s_in)
+            comp.wait_event(ev_in[b])
+            comp.wait_event(ev_out[b])
+            for p_ in prep:
+                check_status(p_())
+            ev_comp[b].record(comp)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                download(b)
+            ev_out[b].record(s_out)
+            if jl == last:
+                comp.wait_stream(s_out)   # the end event follows the last download
+        return [one]
+
+    ms_s = ctx.timed(serial_calls, K, W, graph_ok=False)
+    if r.errors() != 0:
+        raise RuntimeError("device error bits set in the end-to-end leg")
+    ctx.launches += K * wl.n_layers
+    tot_s = ctx.reduce_max(ms_s)
+    serial = {"value": whole_job_rate(wl.units_per_step * K, ctx.world, tot_s), "unit": UNIT,
+              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_s / K,
+              "copies": a.e2e_copies,
+              "path": f"one stream: {copies} -> dl_decode_step per layer -> {copies_out}, "
+                      "step after step, all inside the events"}
+    if a.l2 != "rotate":
+        return {"e2e": serial}
+    ms_p = ctx.timed(piped_calls, K, W, graph_ok=False)
+    if r.errors() != 0:
+        raise RuntimeError("device error bits set in the end-to-end leg")
+    ctx.launches += K * wl.n_layers
+    tot_p = ctx.reduce_max(ms_p)
+    e2e = {"value": whole_job_rate(wl.units_per_step * K, ctx.world, tot_p), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": tot_p / K,
+           "copies": a.e2e_copies,
+           "path": f"{copies} (copy stream) -> dl_decode_step per layer (compute "
+                   f"stream) -> {copies_out} (second copy stream), double-buffered so "
+                   "that step j+1's upload and step j-1's download overlap step j's "
+                   "kernels; every copy inside the events"}
+    return {"e2e": e2e, "e2e_serial": serial}
+
+
+def run_gpu(a, wl, rank, world, dist):
+    ctx = GpuContext(a, world, dist)
+    K, W = a.steps, a.warmup
+    rec, kept = measure_decode(ctx, wl, K, W, keep=not a.no_e2e)
+    launches_headline = K * wl.n_layers
+    result = {"value": rec["value"], "ms_per_step": rec["ms_per_step"], "roofline": rec["roofline"],
+              "gpu_launches": launches_headline, "rotation_groups": rec["rotation_groups"],
+              "live_entries": rec["live_entries"], "deferred_bytes_per_step": rec["deferred_bytes_per_step"]}
+    for k in ("eager", "deferred_over_eager", "eager_bytes_over_deferred"):
+        if k in rec:
+            result[k] = rec[k]
+    if kept is not None:
+        r, setup, R, goffs = kept
+        result.update(measure_e2e(ctx, wl, K, W, r, setup, R, goffs))
+        del r, setup, kept
+        ctx.torch.cuda.empty_cache()
+    subs = []
+    for swl in spec_list(a.subs):
+        Ks = sub_steps(swl, K, a.log_format)
+        srec, _ = measure_decode(ctx, swl, Ks, max(W, 3))
+        subs.append(srec)
+    if subs:
+        result["subs"] = subs
+    merges = []
+    for mwl in spec_list(a.merge_legs):
+        merges.append(measure_merge(ctx, mwl, max(K, 4), max(W, 2)))
+    if merges:
+        result["merge_legs"] = merges
+    result["gpu_launches_all_legs"] = ctx.launches
+    result["graph_uploaded"] = ctx.graph_uploaded
+    result["clocks"] = ctx.sampler.stop()
     return result
 
 
@@ -703,7 +1011,7 @@ def run_reference(a, wl):
                                          int(probe * budget_s / max(1, a.steps + a.warmup))))
     n_rows = max(1, min(wl.batch, per_step_heads // wl.n_heads))
     rows = rows_all[:n_rows]
-    S = synth.initial_state(wl, 0)[rows].astype(np.float64)
+    S = synth.initial_state(wl.with_(batch=n_rows), 0).astype(np.float64)
     x = synth.step_inputs(wl, 0, 0)
     xs = synth.select_rows(wl, x, rows)
     f = lambda k: synth.input_to_f64(xs[k], wl.in_dtype)[None]
@@ -730,20 +1038,23 @@ def run_reference(a, wl):
             "device": f"host CPU, {threads} threads (no GPU)",
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * sum(times) / a.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch, a.log_format, a.replay),
+            "data": "synthetic", "config": config_of(wl, 1, a.tile_v, a.l2, a.launch, a.log_format, a.replay,
+                                                     a.phases),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-def main():
-    a = parse()
+def main(argv=None):
+    a = parse(argv)
     sys.path.insert(0, ROOT)
     wl = workload(a)
     if a.traffic_from:
-        key = config_of(wl, 1, log_format=a.log_format)["workload"]
-        text = traffic_summary_from_ncu(a.traffic_from, key, r"warp_head_kernel|step_kernel")
-        open(PROFILE_TRAFFIC, "w").write(text)
+        kern = {"decode": r"warp_head_kernel|step_kernel", "eager": r"step_kernel",
+                "merge": r"merge_kernel", "materialize": r"merge_kernel"}[a.traffic_kind]
+        text = traffic_summary_from_ncu(a.traffic_from, workload_key(wl, a.log_format), kern, a.traffic_kind)
+        with open(PROFILE_TRAFFIC, "a") as f:
+            f.write(text + "\n")
         print(text)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -777,11 +1088,12 @@ def main():
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; bf16 q/k/v, fp32 lambda/beta, fp32 state and log)",
-            "config": config_of(wl, world, a.tile_v, a.l2, a.launch, a.log_format, a.replay), "roofline": res["roofline"],
-            "gpu_launches": res["gpu_launches"],
+            "config": config_of(wl, world, a.tile_v, a.l2, a.launch, a.log_format, a.replay, a.phases),
+            "roofline": res["roofline"], "gpu_launches": res["gpu_launches"],
             "hbm_tbs": res["roofline"]["achieved"] / 1e3}
-    for k in ("eager", "deferred_bytes_per_step", "e2e", "e2e_serial", "clocks", "rotation_groups",
-              "graph_uploaded"):
+    for k in ("live_entries", "eager", "deferred_over_eager", "eager_bytes_over_deferred",
+              "deferred_bytes_per_step", "e2e", "e2e_serial", "clocks", "rotation_groups",
+              "graph_uploaded", "subs", "merge_legs", "gpu_launches_all_legs"):
         if k in res:
             line[k] = res[k]
     if world == 1 and not a.no_cpu:

@@ -11,9 +11,11 @@ the common steps, slot b takes ``offsets[b]`` decode steps with its own pre-step
 inputs, so slots reach their merge steps at different times.
 
 Slot groups: with ``n_groups = R > 1`` the pool holds R disjoint copies of the
-batch's slots (group g uses ids ``g * per_group + slots``), each prefilled and
-staggered the same way.  Stepping the groups in turn gives a working set R times
-one step's, for timing a batch whose own state fits in L2 without an L2 flush.
+batch's slots (group g uses ids ``g * per_group + slots``), each prefilled the
+same way and staggered by its own row of ``offsets`` (the workload's offsets for
+every group unless given).  Stepping the groups in turn gives a working set R
+times one step's, for timing a batch whose own state fits in L2 without an L2
+flush.
 """
 from __future__ import annotations
 
@@ -36,7 +38,7 @@ class DecodeRunner:
     def __init__(self, wl: synth.Workload, *, n_slots: int | None = None, slot_seed: int | None = None,
                  layers=None, mode: str = "deferred", update: str | None = None,
                  device: str = "cuda", tile_v: int = 0, n_groups: int = 1, log_format: str = "fp32",
-                 replay: str = "per_tile"):
+                 replay: str = "per_tile", offsets=None):
         if mode not in ("deferred", "eager"):
             raise ValueError(mode)
         self.wl = wl
@@ -60,14 +62,38 @@ class DecodeRunner:
                             device=device, with_log=(mode == "deferred"), tile_v=tile_v,
                             log_format=log_format, replay=replay)
         self.offsets = synth.slot_offsets(wl)
+        # per-group staggering offsets [n_groups, batch]
+        if offsets is None:
+            self.group_offsets = np.tile(self.offsets, (n_groups, 1))
+        else:
+            go = np.asarray(offsets, dtype=np.int64)
+            if go.shape != (n_groups, wl.batch) or (go < 0).any():
+                raise ValueError("offsets must be non-negative with shape [n_groups, batch]")
+            self.group_offsets = go
+            self.offsets = go[0]
 
     # -- set-up ----------------------------------------------------------------
-    def load_initial_state(self):
-        """Prefill: write each slot's initial state into the base, empty its log."""
+    def load_initial_state(self, on_device: bool = False):
+        """Prefill: write each slot's initial state into the base, empty its log.
+
+        on_device: draw N(0, init_std^2) states with torch's seeded device generator
+        instead of synth.initial_state (much faster for multi-GB pools; the values
+        then differ from the oracle's, so this is for timing only)."""
         for layer in self.layers:
-            S0 = torch.from_numpy(synth.initial_state(self.wl, layer)).to(self.device)
+            if on_device:
+                shape = (self.wl.batch, self.wl.n_heads, self.wl.d_k, self.wl.d_v)
+                if self.wl.init_std == 0.0:
+                    S0 = torch.zeros(shape, dtype=torch.float32, device=self.device)
+                else:
+                    g = torch.Generator(device=self.device)
+                    g.manual_seed(self.wl.seed * 1000 + layer)
+                    S0 = torch.randn(shape, generator=g, dtype=torch.float32, device=self.device)
+                    S0.mul_(self.wl.init_std)
+            else:
+                S0 = torch.from_numpy(synth.initial_state(self.wl, layer)).to(self.device)
             for gs in self.group_slots:
                 self.pool.state[gs.long(), layer] = S0
+            del S0
         for gs in self.group_slots:
             dl.dl_reset_slots(self.pool, gs)
 
@@ -89,16 +115,40 @@ class DecodeRunner:
         return fn(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"],
                   out=out, lambda_per_head=self.wl.lambda_const, stream=stream)
 
-    def run_presteps(self):
-        """Staggering: slot b takes offsets[b] untimed decode steps first."""
-        n = int(self.offsets.max()) if len(self.offsets) else 0
+    def run_presteps(self, inputs=None):
+        """Staggering: slot b of group g takes group_offsets[g, b] untimed decode steps
+        first.  inputs(p, layer) -> device inputs of the whole batch for pre-step p
+        (default: the workload's own seeded pre-step inputs)."""
+        go = self.group_offsets
+        n = int(go.max()) if go.size else 0
         for p in range(n):
-            rows = np.nonzero(self.offsets > p)[0]
-            sel = torch.from_numpy(rows).to(self.device)
             for layer in self.layers:
-                x = self.device_inputs(synth.step_inputs(self.wl, p, layer, prestep=True), rows)
-                for gs in self.group_slots:
+                if inputs is None:
+                    xh = synth.step_inputs(self.wl, p, layer, prestep=True)
+                x_all = None
+                for g, gs in enumerate(self.group_slots):
+                    rows = np.nonzero(go[g] > p)[0]
+                    if len(rows) == 0:
+                        continue
+                    if inputs is None:
+                        x = self.device_inputs(xh, rows)
+                    else:
+                        if x_all is None:
+                            x_all = inputs(p, layer)
+                        x = self.select_device_rows(x_all, rows)
+                    sel = torch.from_numpy(rows).to(self.device)
                     self.call(layer, x, slots=gs[sel])
+
+    def select_device_rows(self, x: dict, rows) -> dict:
+        """Rows of a device input dict (a per-head constant lambda is kept whole)."""
+        idx = torch.as_tensor(np.asarray(rows), device=self.device, dtype=torch.long)
+        out = {}
+        for k, v in x.items():
+            if v is None or (k == "lam" and self.wl.lambda_const):
+                out[k] = v
+            else:
+                out[k] = v.index_select(0, idx).contiguous()
+        return out
 
     def materialize(self, layer: int) -> torch.Tensor:
         if self.mode == "eager":

@@ -153,3 +153,86 @@ def test_packed_step_inputs(wl):
                           rc(layer["beta"]), rc(o["o"]), wl.lambda_const)
         assert a.q == layer["q"].data_ptr() and a.v == layer["v"].data_ptr()
         assert a.out == o["o"].data_ptr()
+
+
+def test_spread_phases_give_every_launch_the_cycle_average():
+    """With spread phases a batch of L or more slots holds each live length equally in
+    every launch, so any window of timed steps is the amortised step."""
+    for wl in (synth.KDA, synth.GLA_DIAG, synth.RETNET.with_(batch=1024, staggered=False)):
+        R = bench.rotation_groups(wl, "rotate")
+        go = bench.phase_offsets(wl, R, "spread")
+        assert go.shape == (R, wl.batch)
+        L = wl.log_cap
+        for first, K in ((0, 1), (5, 20), (3, 7)):
+            b, hist = bench.timed_window_bytes(wl, go, first, K)
+            assert (hist == hist[0]).all() and hist.sum() == K * wl.batch
+            per = b / (K * wl.units_per_step)
+            assert per == pytest.approx(traffic.deferred_cycle_average(wl))
+        assert L - 1 in set(bench.group_live_entries(go, 0, L))
+
+
+def test_spread_phases_continue_across_groups_for_small_batches():
+    """Batch 1 (GDN): launch j holds live length (j + j // R) mod L, so consecutive
+    launches walk the merge cycle and L of them cover it once."""
+    wl = synth.GDN_GVA
+    R = bench.rotation_groups(wl, "rotate")
+    go = bench.phase_offsets(wl, R, "spread")
+    L = wl.log_cap
+    for j in range(3 * R):
+        assert bench.group_live_entries(go, j, L)[0] == (j % R + j // R) % L
+    _, hist = bench.timed_window_bytes(wl, go, 0, L)
+    assert (hist == 1).all()
+
+
+def test_staggered_workload_keeps_its_own_offsets_in_group_zero():
+    wl = synth.RETNET.with_(batch=64)
+    go = bench.phase_offsets(wl, 3, "spread")
+    np.testing.assert_array_equal(go[0], synth.slot_offsets(wl))
+    np.testing.assert_array_equal(go[1], (synth.slot_offsets(wl) + 64) % wl.log_cap)
+    np.testing.assert_array_equal(bench.phase_offsets(wl, 3, "workload"), np.tile(synth.slot_offsets(wl), (3, 1)))
+    # group_live_entries with equal offsets per group is the single-offset rule
+    for j in range(20):
+        np.testing.assert_array_equal(bench.group_live_entries(np.tile(synth.slot_offsets(wl), (3, 1)), j, 32),
+                                      bench.live_entries(synth.slot_offsets(wl), j, 3, 32))
+
+
+def test_sub_record_steps_and_specs():
+    for spec in bench.DEFAULT_SUBS.split(","):
+        wl = bench.parse_spec(spec)
+        n = bench.sub_steps(wl, 20)
+        assert n >= 20 and n % wl.log_cap == 0 and n <= bench.SUB_MAX_STEPS
+    wl = bench.parse_spec("gla_rwkv6_diag:b64:L8")
+    assert (wl.batch, wl.log_cap) == (64, 8)
+    assert bench.parse_spec("retnet_scalar:b1024").batch == 1024
+    with pytest.raises(SystemExit):
+        bench.parse_spec("nope")
+    with pytest.raises(SystemExit):
+        bench.parse_spec("kda_diag_delta:x3")
+    assert bench.spec_list("none") == []
+    assert bench.parse(["--steps", "20"]).workload == "kda_diag_delta"
+
+
+def test_distinct_steps_bounds_host_generation():
+    for wl in (synth.KDA, synth.RETNET.with_(batch=1024), synth.GLA_DIAG, synth.GDN_GVA):
+        n = bench.distinct_steps(wl)
+        assert 2 <= n <= max(2, wl.steps)
+        assert n == 2 or n * traffic.token_bytes(wl) * wl.units_per_step <= bench.HOST_INPUT_BYTES
+
+
+def test_config_names_the_delta_reading():
+    cfg = bench.config_of(synth.KDA, 1)
+    assert "decayed" in cfg["delta_reading"] and cfg["workload"] == "kda_diag_delta_b256_h32_d128_L16"
+    assert "delta_reading" not in bench.config_of(synth.GLA_DIAG, 1)
+
+
+def test_traffic_records_by_kind(tmp_path, monkeypatch):
+    p = tmp_path / "t.txt"
+    sha = bench.kernel_source_hash()
+    p.write_text(f"workload = w\nkind = decode\nkernel_sha = {sha}\ndram_bytes_per_launch = 10\n\n"
+                 f"workload = w\nkind = eager\nkernel_sha = {sha}\ndram_bytes_per_launch = 20\n"
+                 f"l2_write_bytes_per_launch = 7\n")
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
+    assert bench.recorded_traffic("w") == 10.0
+    assert bench.recorded_traffic("w", "eager") == 20.0
+    assert bench.recorded_traffic("w", "eager", "l2_write_bytes_per_launch") == 7.0
+    assert bench.recorded_traffic("w", "merge") is None
