@@ -247,9 +247,28 @@ dl_status dl_reset_slots(dl_pool *pool, const int32_t *slots, int32_t batch, voi
 dl_status dl_materialize(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
                          float *dense_out, void *stream);
 
-/* Synchronise `stream`, copy the device error word to *bits, and clear it when
- * `clear` is non-zero.  Returns DL_ERR_DEVICE when any bit was set. */
+/* Synchronise `stream`, copy the device error word to *bits, and, when `clear` is
+ * non-zero, clear the bits just read (an atomic AND on the device, ordered on
+ * `stream`, then a second synchronisation): a bit that a kernel on another stream
+ * sets between the copy and the clear stays set for the next read.  Returns
+ * DL_ERR_DEVICE when any bit was set.
+ *
+ * After any bit is reported, prefill and reset (dl_reset_slots) the affected slots
+ * before their next step.  A skipped work item leaves its slot as it was, but a
+ * kernel that abandoned a call (DL_EBIT_TIMEOUT) can leave a slot's base, log and
+ * arrival counters part-way through the step. */
 dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *stream);
+
+/* Fault injection for tests (the paper has no counterpart).  Sets, process-wide,
+ * the time limit of the whole-head decode kernel's pipeline waits (a bulk copy's
+ * arrival, a split merge head's partial output) for launches issued after the
+ * call; limit_ns <= 0 restores the default of 100 ms.  A short limit makes waits
+ * run out: the kernel then sets DL_EBIT_TIMEOUT, stops the affected work, waits
+ * with the default 100 ms bound for its own bulk copies still in flight, frees its
+ * tensor memory and returns, so the context stays usable.  The slots of such a
+ * call must then be prefilled and reset (see dl_read_error).  Always DL_OK; makes
+ * no CUDA call. */
+dl_status dl_debug_wait_limit(int64_t limit_ns);
 
 /* Decode step that allocates nothing.  The paper has no counterpart: this entry
  * point exists for integration only.
@@ -276,9 +295,10 @@ dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *strea
  *  - All calls share that one array.  Each call first clears the counters it uses
  *    (an asynchronous memset on `stream`), so calls that overlap on the GPU (two
  *    streams, or two host threads) race; issue them in order on one stream.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, which can load the module).  Make that first call
- *    before any stream capture.
+ *  - Every call looks up the array's address in the current device's context
+ *    (cudaGetSymbolAddress; nothing is cached between calls).  The first lookup on
+ *    a device can load the module, so make the first call on each device before
+ *    any stream capture.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine. */
 #define DL_NOALLOC_MAX_COUNTERS 65536
 dl_status dl_decode_step_noalloc(const dl_pool_desc *desc, int32_t layer,

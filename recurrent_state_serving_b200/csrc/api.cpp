@@ -1,6 +1,7 @@
 // C ABI of the base + log recurrent-state decode library: argument validation,
 // launch-shape selection and error reporting.  The arithmetic lives in the
 // kernels (dl_kernels.cuh); nothing here computes on the host.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -17,6 +18,9 @@ struct dl_pool {
 };
 
 namespace {
+
+constexpr unsigned long long kDefaultWaitNs = 100000000ull;  // 100 ms
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -66,6 +70,7 @@ dl::KParams base_params(const dl_pool_desc &d, int layer) {
     p.b16 = l.b16;
     p.layer = layer;
     p.cl = 1;
+    p.wait_ns = dl::wait_limit_ns();
     return p;
 }
 
@@ -278,12 +283,18 @@ DL_API dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void
         return DL_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return DL_ERR_CUDA;
     if (clear && host) {
-        if (cudaMemsetAsync(pool->d.err_word, 0, sizeof(int32_t), st) != cudaSuccess)
-            return DL_ERR_CUDA;
+        // clear only the bits just read, atomically: a bit another stream's kernel
+        // sets in the meantime stays set for the next read
+        if (dl::launch_clear_bits(pool->d.err_word, host, st) != cudaSuccess) return DL_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return DL_ERR_CUDA;
     }
     *bits = host;
     return host ? DL_ERR_DEVICE : DL_OK;
+}
+
+DL_API dl_status dl_debug_wait_limit(int64_t limit_ns) {
+    g_wait_ns.store(limit_ns > 0 ? (unsigned long long)limit_ns : kDefaultWaitNs);
+    return DL_OK;
 }
 
 DL_API const char *dl_status_string(dl_status status) {
@@ -300,6 +311,8 @@ DL_API const char *dl_status_string(dl_status status) {
 }
 
 namespace dl {
+
+unsigned long long wait_limit_ns() { return g_wait_ns.load(); }
 
 // Checks a bare descriptor with the rules of dl_create_pool, except that its
 // arrival-counter buffer is not looked at (the entry point that allocates nothing

@@ -41,7 +41,12 @@ struct KParams {
     int eager;       // eager step: c = 0 and always write back, no log
     int want_out;    // write o_t
     int undecayed;   // delta correction from S_{t-1} instead of Diag(e^lambda) S_{t-1}
+    unsigned long long wait_ns;  // bound on the whole-head kernel's pipeline waits
 };
+
+// Bound of the kernels' pipeline waits (ns) for launches issued now: 100 ms unless
+// a test shortened it with dl_debug_wait_limit.
+unsigned long long wait_limit_ns();
 
 // Value-tile width chosen for a launch (16 or 32 columns).
 int pick_bv(int dk, int dv, long long work_items_at_32);
@@ -57,6 +62,8 @@ cudaError_t launch_merge(const KParams &p, int bv, int decay, bool materialize,
                          cudaStream_t st);
 cudaError_t launch_reset(const int32_t *slots, int batch, int n_slots, int n_layers,
                          int32_t *log_len, int32_t *arrive, int32_t *err, cudaStream_t st);
+// Atomically clears `bits` in the error word (bits set meanwhile by other launches survive).
+cudaError_t launch_clear_bits(int32_t *err, int32_t bits, cudaStream_t st);
 
 // Floats of dynamic shared memory a launch needs.
 inline size_t dyn_floats(int L, int dk, int bv, bool need_A) {

@@ -53,9 +53,10 @@
 // programmatic stream serialization: a CTA sets up its mbarriers and TMEM while the
 // previous kernel in the stream finishes, and reads global memory only after it.
 //
-// Every wait is bounded (100 ms); a warp whose wait runs out sets
-// DL_EBIT_TIMEOUT, stops, and waits (bounded again) for its own copies still in
-// flight before the CTA frees its tensor memory and exits.
+// Every wait is bounded (p.wait_ns, 100 ms unless a test shortens it); a warp whose
+// wait runs out sets DL_EBIT_TIMEOUT, stops, and waits (bounded by the fixed 100 ms
+// WAIT_NS, whatever p.wait_ns is) for its own copies still in flight before the
+// CTA frees its tensor memory and exits.
 #pragma once
 
 #include "dl_kernels.cuh"
@@ -74,7 +75,7 @@ constexpr int NTHREADS = NW * 32;
 constexpr int NSW = 3;                      // stages per warp
 constexpr int RPB = 4;                      // log entries per load block (merge rounds)
 constexpr int MRB = CF / (DK + DV);         // entries per merge round (A' and b in one stage)
-constexpr uint64_t WAIT_NS = 100000000ull;  // bound on every wait
+constexpr uint64_t WAIT_NS = 100000000ull;  // bound on the abort path's drain waits
 constexpr int NB = NSW + 2;                 // mbarriers per warp: stream stages + merge re-stream
 constexpr int TM_ENT = 32;                  // merge entries staged in TMEM per warp
 constexpr uint32_t TM_COLS = 512;           // TMEM columns per CTA (all of them)
@@ -406,7 +407,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     };
     // wait for stream position gc; false when the wait ran out (warp-uniform)
     auto wait_chunk = [&]() -> bool {
-        const bool ok = ptx::mbar_wait_bounded(&fb[gc % NSW], (gc / NSW) & 1, WAIT_NS);
+        const bool ok = ptx::mbar_wait_bounded(&fb[gc % NSW], (gc / NSW) & 1, p.wait_ns);
         return __all_sync(FULL, ok);
     };
     // done reading stream position gc: free its stage and keep the ring full
@@ -687,7 +688,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     if (lane == 0) {
                         const uint64_t t0 = ptx::globaltimer_ns();
                         while (!(ready = (atomicAdd(cm, 0) & 4) != 0)) {
-                            if (ptx::globaltimer_ns() - t0 > WAIT_NS) break;
+                            if (ptx::globaltimer_ns() - t0 > p.wait_ns) break;
                         }
                     }
                     ready = __shfl_sync(FULL, ready ? 1 : 0, 0) != 0;
@@ -780,7 +781,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     __syncwarp();
                     for (int cx = 0; cx < NCH; ++cx) {
                         const uint32_t bb = cx & 1;
-                        const bool ok = ptx::mbar_wait_bounded(&pb[bb], (pph >> bb) & 1u, WAIT_NS);
+                        const bool ok = ptx::mbar_wait_bounded(&pb[bb], (pph >> bb) & 1u, p.wait_ns);
                         if (!__all_sync(FULL, ok)) { abort = true; break; }
                         pph ^= 1u << bb;
                         pb_pend &= ~(1u << bb);

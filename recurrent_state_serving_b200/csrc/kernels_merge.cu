@@ -60,7 +60,14 @@ __global__ void reset_kernel(const int32_t *slots, int batch, int n_slots, int n
     arrive[(size_t)s * n_layers + l] = 0;
 }
 
+__global__ void clear_bits_kernel(int32_t *err, int32_t bits) { atomicAnd(err, ~bits); }
+
 }  // namespace
+
+cudaError_t launch_clear_bits(int32_t *err, int32_t bits, cudaStream_t st) {
+    clear_bits_kernel<<<1, 1, 0, st>>>(err, bits);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_merge(const KParams &p, int bv, int decay, bool materialize, cudaStream_t st) {
     if (p.dk == 16 && bv == 16) return merge_decay<16, 16>(p, decay, materialize, st);

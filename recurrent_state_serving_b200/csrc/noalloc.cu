@@ -23,23 +23,16 @@ namespace {
 // this array (DL_NOALLOC_MAX_COUNTERS * 4 bytes) until the process exits.
 static __device__ __align__(256) int32_t g_arrive_scratch[DL_NOALLOC_MAX_COUNTERS];
 
-constexpr int kMaxDevices = 64;
-int32_t *g_scratch_addr[kMaxDevices];  // device address of the array, per device
-
-// Device address of g_arrive_scratch on the current device.  In host code the
-// array's name only stands in for the symbol, so the address is resolved once
-// per device with cudaGetSymbolAddress (which may load the module: keep the
-// first call out of stream capture).
+// Device address of g_arrive_scratch in the current device's context.  In host code
+// the array's name only stands in for the symbol, so the address is looked up with
+// cudaGetSymbolAddress on every call: nothing is cached, so no host-side state is
+// shared between threads and no address outlives a context torn down and made again.
+// The first lookup on a device can load the module, so that first call belongs
+// outside stream capture.
 dl_status scratch_on_current_device(int32_t **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DL_ERR_CUDA;
-    if (!g_scratch_addr[dev]) {
-        void *addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_arrive_scratch) != cudaSuccess || !addr)
-            return DL_ERR_CUDA;
-        g_scratch_addr[dev] = static_cast<int32_t *>(addr);
-    }
-    *out = g_scratch_addr[dev];
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_arrive_scratch) != cudaSuccess || !addr) return DL_ERR_CUDA;
+    *out = static_cast<int32_t *>(addr);
     return DL_OK;
 }
 

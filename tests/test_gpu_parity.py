@@ -423,3 +423,43 @@ def test_split_merge_heads_match_the_oracle(staggered, log_format):
     oe, se, _ = H.gpu_rollout(re_, T, ckpts=[T])
     H.check_steps(outs[0], oe[0], tol=H.REL_L2_GPU, elem=None, what="deferred vs eager")
     H.check_steps(states[0], se[0], tol=H.REL_L2_GPU, elem=None, what="state")
+
+
+def test_expired_wait_sets_the_timeout_bit_and_the_pool_recovers():
+    """A pipeline wait of the whole-head kernel made to run out (test hook: a 1 ns
+    limit) sets DL_EBIT_TIMEOUT; the kernel drains its own copies and returns, the
+    context stays usable, and after a fresh prefill and reset the same pool matches
+    the oracle again."""
+    wl = synth.GLA_DIAG.with_(batch=16, n_heads=16, n_kheads=16, steps=12, log_cap=4)
+    r = DecodeRunner(wl, tile_v=128)
+    r.load_initial_state()
+    dl.dl_debug_wait_limit(1)
+    try:
+        for t in range(2 * wl.log_cap):   # append steps and merge steps
+            r.call(0, r.gen_inputs(t, 0))
+        bits = dl.dl_read_error(r.pool, clear=False)
+    finally:
+        dl.dl_debug_wait_limit(0)
+    assert bits & dl.DL_EBIT_TIMEOUT, f"error bits {bits:#x}"
+    assert dl.dl_read_error(r.pool, clear=True) == bits      # read, then cleared
+    assert dl.dl_read_error(r.pool) == 0
+    # ordinary calls on the same pool after prefill and reset
+    T = wl.steps
+    outs, states, _ = H.gpu_rollout(r, T, ckpts=[T])
+    assert r.errors() == 0
+    O, S = H.oracle_reference(wl, 0, T, ckpts=[T])
+    H.check_steps(outs[0], O, what="output after recovery")
+    H.check_steps(states[0], S, elem=None, what="state after recovery")
+
+
+def test_read_error_clears_only_when_asked():
+    wl = synth.GLA_DIAG.with_(batch=2, n_heads=2, n_kheads=2, steps=1)
+    r = DecodeRunner(wl, n_slots=4)
+    r.load_initial_state()
+    x = r.gen_inputs(0, 0)
+    bad = torch.tensor([0, 99], dtype=torch.int32, device="cuda")
+    dl.dl_decode_step(r.pool, 0, bad, x["q"], x["k"], x["v"], lam=x["lam"])
+    assert dl.dl_read_error(r.pool, clear=False) == dl.DL_EBIT_SLOT_RANGE
+    assert dl.dl_read_error(r.pool, clear=False) == dl.DL_EBIT_SLOT_RANGE
+    assert dl.dl_read_error(r.pool, clear=True) == dl.DL_EBIT_SLOT_RANGE
+    assert dl.dl_read_error(r.pool, clear=False) == 0
