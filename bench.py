@@ -100,6 +100,9 @@ def parse(argv=None):
                     help="comma list of name[:bB][:LL] workloads whose dl_merge/dl_materialize are timed, or 'none'")
     ap.add_argument("--phases", default="spread", choices=["spread", "workload"],
                     help="slot merge phases: spread over each launch, or the workload's own offsets")
+    ap.add_argument("--merge", default="adaptive", choices=["adaptive", "capacity"],
+                    help="dl_decode_step merge policy: adaptive (launches too small to fill the GPU "
+                         "merge every step) or capacity (every slot merges on its L-th step)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -196,17 +199,23 @@ def group_live_entries(group_offsets, step_index: int, log_cap: int):
     return (group_offsets[step_index % R] + step_index // R) % log_cap
 
 
-def timed_window_bytes(wl, group_offsets, first: int, K: int, log_format: str = "fp32"):
+def timed_window_bytes(wl, group_offsets, first: int, K: int, log_format: str = "fp32",
+                       merge_every: bool = False):
     """Algorithmic bytes of global steps first .. first+K-1 (all layers and heads)
-    and the histogram of the slots' live entries at those steps."""
+    and the histogram of the slots' live entries at those steps.  merge_every: the
+    launches merge every slot on every step (the adaptive policy on a small launch),
+    so every slot enters with an empty log and takes the merge step."""
     from recurrent_state_serving_b200 import traffic
     L = wl.log_cap
-    per_c = [traffic.deferred_head_step(wl, c, merge=(c == L - 1), log_format=log_format) for c in range(L)]
+    scale = wl.n_heads * wl.n_layers
     hist = np.zeros(L, np.int64)
+    if merge_every:
+        hist[0] = K * wl.batch
+        return hist[0] * traffic.deferred_head_step(wl, 0, merge=True, log_format=log_format) * scale, hist
+    per_c = [traffic.deferred_head_step(wl, c, merge=(c == L - 1), log_format=log_format) for c in range(L)]
     for j in range(first, first + K):
         hist += np.bincount(group_live_entries(group_offsets, j, L), minlength=L)
     per_slot = float(np.dot(hist, per_c))
-    scale = wl.n_heads * wl.n_layers
     return per_slot * scale, hist
 
 
@@ -617,7 +626,7 @@ class WorkloadSetup:
         return self.dev[p % self.ndist][layer]
 
 
-def prepared_calls(kind, wl, runner, setup, R, cache):
+def prepared_calls(kind, wl, runner, setup, R, cache, merge="capacity"):
     """Step j: group j mod R, distinct inputs j mod ndist (argument blocks built once)."""
     from recurrent_state_serving_b200 import deltalog as dl
 
@@ -626,7 +635,8 @@ def prepared_calls(kind, wl, runner, setup, R, cache):
         if key not in cache:
             g, t = key
             cache[key] = [dl.PreparedStep(kind, runner.pool, l, runner.group_slots[g], x["q"], x["k"],
-                                          x["v"], x["lam"], x["beta"], setup.outs[l], wl.lambda_const)
+                                          x["v"], x["lam"], x["beta"], setup.outs[l], wl.lambda_const,
+                                          auto_merge=merge)
                           for l, x in enumerate(setup.dev[t])]
         return [(lambda p=p: check_status(p())) for p in cache[key]]
     return calls
@@ -642,39 +652,63 @@ def roofline_record(achieved_gbs, kernel, launches, total_ms, bytes_per_launch, 
             "frac_of_8tbs_spec": round(achieved_gbs / 8000.0, 4)}
 
 
-def measure_decode(ctx, wl, K, W, *, eager=True, keep=False):
-    """Deferred decode steps of a workload (the product path), then the in-library
-    eager step on the same workload.  Returns (record, runner and setup when keep)."""
+def decode_leg(ctx, wl, K, W, setup, merge):
+    """Timed deferred decode steps under one merge policy.  Returns (record, runner,
+    rotation groups, group offsets)."""
+    from recurrent_state_serving_b200 import deltalog as dl
     from recurrent_state_serving_b200 import traffic
     from recurrent_state_serving_b200.runner import DecodeRunner
-    torch = ctx.torch
     a = ctx.a
-    setup = WorkloadSetup(ctx, wl)
     R = rotation_groups(wl, a.l2)
     goffs = phase_offsets(wl, R, a.phases)
     r = DecodeRunner(wl, device=str(ctx.dev), tile_v=a.tile_v, n_groups=R, log_format=a.log_format,
-                     replay=a.replay, offsets=goffs)
+                     replay=a.replay, offsets=goffs, merge=merge)
+    every = dl.dl_merge_policy(wl.batch, wl.n_heads, merge)
     r.load_initial_state(on_device=True)
     r.run_presteps(inputs=setup.prestep_inputs)
-    total_ms = ctx.timed(prepared_calls("decode", wl, r, setup, R, {}), K, W)
+    total_ms = ctx.timed(prepared_calls("decode", wl, r, setup, R, {}, merge), K, W)
     if r.errors() != 0:
         raise RuntimeError("device error bits set during the benchmark")
     max_ms = ctx.reduce_max(total_ms)
     launches = K * wl.n_layers
     ctx.launches += launches
-    bytes_total, hist = timed_window_bytes(wl, goffs, W, K, a.log_format)
+    bytes_total, hist = timed_window_bytes(wl, goffs, W, K, a.log_format, merge_every=every)
     achieved = bytes_total / (total_ms / 1e3) / 1e9
     key = workload_key(wl, a.log_format)
     units = hist.sum() * wl.n_heads * wl.n_layers
-    rec = {"workload": key, "value": whole_job_rate(wl.units_per_step * K, ctx.world, max_ms), "unit": UNIT,
+    kernel = "dl::step_kernel (merging every step)" if every else res_kernel_name(wl, a.tile_v)
+    rec = {"workload": key, "merge_policy": merge, "merges_every_step": every,
+           "value": whole_job_rate(wl.units_per_step * K, ctx.world, max_ms), "unit": UNIT,
            "ms_per_step": max_ms / K, "steps": K, "warmup": W, "rotation_groups": R,
-           "roofline": roofline_record(achieved, res_kernel_name(wl, a.tile_v), launches, total_ms,
-                                       bytes_total / launches, recorded_traffic(key, "decode")),
+           "roofline": roofline_record(achieved, kernel, launches, total_ms,
+                                       bytes_total / launches,
+                                       None if every else recorded_traffic(key, "decode")),
            "live_entries": {"hist": [int(x) for x in hist],
-                            "merge_share": round(float(hist[-1]) / max(1, hist.sum()), 4),
+                            "merge_share": 1.0 if every else round(float(hist[-1]) / max(1, hist.sum()), 4),
                             "bytes_per_head_step": round(bytes_total / units, 1),
                             "cycle_average_model": round(traffic.deferred_cycle_average(wl, a.log_format), 1)},
            "deferred_bytes_per_step": round(bytes_total / K)}
+    return rec, r, R, goffs
+
+
+def measure_decode(ctx, wl, K, W, *, eager=True, keep=False):
+    """Deferred decode steps of a workload (the product path, merge policy --merge),
+    then the in-library eager step on the same workload; when the adaptive policy
+    merges every step (a small launch), also the at-capacity policy.  Returns
+    (record, runner and setup when keep)."""
+    from recurrent_state_serving_b200 import traffic
+    from recurrent_state_serving_b200.runner import DecodeRunner
+    torch = ctx.torch
+    a = ctx.a
+    setup = WorkloadSetup(ctx, wl)
+    rec, r, R, goffs = decode_leg(ctx, wl, K, W, setup, a.merge)
+    key = rec["workload"]
+    bytes_total = rec["deferred_bytes_per_step"] * K
+    launches = K * wl.n_layers
+    if rec["merges_every_step"]:
+        cap, r_cap, _, _ = decode_leg(ctx, wl, K, W, setup, "capacity")
+        rec["at_capacity"] = {k: cap[k] for k in ("value", "ms_per_step", "roofline", "live_entries")}
+        del r_cap
     if wl.update == "delta":
         rec["delta_reading"] = DELTA_READING
     if eager and not a.no_eager:
@@ -836,7 +870,8 @@ def measure_e2e(ctx, wl, K, W, runner, setup, R, goffs):
             for l in range(wl.n_layers):
                 out_host[b][l].copy_(outs_e[b][l], non_blocking=True)
     prep_2 = [[[dl.PreparedStep("decode", r.pool, l, gs, s_["q"], s_["k"], s_["v"], s_["lam"],
-                                s_["beta"], outs_e[b][l], wl.lambda_const) for l, s_ in enumerate(stage[b])]
+                                s_["beta"], outs_e[b][l], wl.lambda_const, auto_merge=r.merge)
+                for l, s_ in enumerate(stage[b])]
                for b in range(2)] for gs in r.group_slots]
     copies = ("one H2D copy of the step's packed pinned inputs" if a.e2e_copies == "packed"
               else "H2D copies of the step's pinned inputs")
@@ -930,8 +965,9 @@ def run_gpu(a, wl, rank, world, dist):
     launches_headline = K * wl.n_layers
     result = {"value": rec["value"], "ms_per_step": rec["ms_per_step"], "roofline": rec["roofline"],
               "gpu_launches": launches_headline, "rotation_groups": rec["rotation_groups"],
-              "live_entries": rec["live_entries"], "deferred_bytes_per_step": rec["deferred_bytes_per_step"]}
-    for k in ("eager", "deferred_over_eager", "eager_bytes_over_deferred"):
+              "live_entries": rec["live_entries"], "deferred_bytes_per_step": rec["deferred_bytes_per_step"],
+              "merge_policy": rec["merge_policy"], "merges_every_step": rec["merges_every_step"]}
+    for k in ("eager", "deferred_over_eager", "eager_bytes_over_deferred", "at_capacity"):
         if k in rec:
             result[k] = rec[k]
     if kept is not None:
@@ -1091,7 +1127,8 @@ def main(argv=None):
             "config": config_of(wl, world, a.tile_v, a.l2, a.launch, a.log_format, a.replay, a.phases),
             "roofline": res["roofline"], "gpu_launches": res["gpu_launches"],
             "hbm_tbs": res["roofline"]["achieved"] / 1e3}
-    for k in ("live_entries", "eager", "deferred_over_eager", "eager_bytes_over_deferred",
+    for k in ("live_entries", "merge_policy", "merges_every_step", "at_capacity", "eager",
+              "deferred_over_eager", "eager_bytes_over_deferred",
               "deferred_bytes_per_step", "e2e", "e2e_serial", "clocks", "rotation_groups",
               "graph_uploaded", "subs", "merge_legs", "gpu_launches_all_legs"):
         if k in res:

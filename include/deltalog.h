@@ -207,20 +207,43 @@ dl_status dl_log_bytes(const dl_pool_desc *desc, int64_t *bytes);
 dl_status dl_create_pool(const dl_pool_desc *desc, dl_pool **out_pool);
 dl_status dl_destroy_pool(dl_pool *pool);
 
+/* Merge policy of dl_decode_step (its auto_merge argument). */
+#define DL_MERGE_NONE 0         /* never merge; a full log is an error                  */
+#define DL_MERGE_AT_CAPACITY 1  /* merge on the slot's log_cap-th step (any other
+                                   non-zero value except DL_MERGE_ADAPTIVE means this)  */
+#define DL_MERGE_ADAPTIVE 2     /* as DL_MERGE_AT_CAPACITY, except that a launch too
+                                   small to fill the GPU merges every slot on every step */
+
 /* One decode step (Section 3.3, AppendDecode + Finalize, and the merge step of
  * the append-merge cycle).  For each slot with c live entries:
- *   c < log_cap - 1, or auto_merge == 0 and c < log_cap:
+ *   c < log_cap - 1, or auto_merge == DL_MERGE_NONE and c < log_cap:
  *       read o_t and, for the delta rule, the correction (Shat^T k_t) off the
  *       read-only base plus the decayed log; append (k_t, b_t, lbar + lambda_t)
  *       as entry c; live length c + 1.
- *   auto_merge != 0 and c >= log_cap - 1 (the slot's merge step):
+ *   auto_merge != DL_MERGE_NONE and c >= log_cap - 1 (the slot's merge step):
  *       compute o_t the same way and write the fully materialised state S_t
  *       (base, log and the token) to the base; live length 0.
- *   auto_merge == 0 and c == log_cap: DL_EBIT_LOG_FULL, slot skipped.
+ *   auto_merge == DL_MERGE_NONE and c == log_cap: DL_EBIT_LOG_FULL, slot skipped.
  * So with auto_merge the merge interval equals log_cap, and log_cap == 1 is
- * the eager recurrence. */
+ * the eager recurrence.
+ *
+ * DL_MERGE_ADAPTIVE: when batch * n_heads is below a few heads per SM of the
+ * current device (dl_merge_policy tells), the launch is latency-bound: its time
+ * is one head's chain of dependent loads plus, on a merge step, that head's
+ * write-back, not the bytes it moves.  Every slot of such a launch then takes the
+ * merge step (folding whatever its log holds), so after the first such step the
+ * launch is the eager recurrence with an empty log, run by the value-tiled kernel.
+ * The outputs and logical states are the same under every policy (the
+ * logical-state equation); only the split between base and log differs. */
 dl_status dl_decode_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
                          int32_t auto_merge, void *stream);
+
+/* Whether dl_decode_step with this batch, head count and auto_merge value merges
+ * every slot on every step (*merges_every_step = 1) on the current device.
+ * DL_ERR_INVALID_ARG for a NULL output, batch < 0 or n_heads <= 0.  Reads the
+ * device's SM count (148 when no device is visible). */
+dl_status dl_merge_policy(int32_t batch, int32_t n_heads, int32_t auto_merge,
+                          int32_t *merges_every_step);
 
 /* Append the step's factors only (no output, never merges).  For the delta rule
  * the base is still read to form b_t.  A full log sets DL_EBIT_LOG_FULL. */

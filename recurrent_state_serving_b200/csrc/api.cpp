@@ -84,16 +84,17 @@ void set_tiles(const dl_pool_desc &d, dl::KParams &p, int batch, int &bv) {
 // kernel streams token rows and writes outputs with 128-bit accesses, so it needs
 // 16-byte aligned q, k, v, per-key lambda and out; calls whose buffers are only
 // element-aligned run the value-tiled kernel.
-bool use_whole_head(const dl_pool_desc &d, const dl_step_args *a, bool want_out, bool eager) {
+bool use_whole_head(const dl_pool_desc &d, const dl_step_args *a, bool want_out, bool rewrites_all) {
     if (!want_out || !dl::whole_head_supported(d.d_k, d.d_v)) return false;
     if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->out, 16))
         return false;
     if (d.decay == DL_DECAY_DIAG && !aligned(a->lambda, 16)) return false;
     if (d.tile_v == 128) return true;
     if (d.tile_v != 0) return false;
-    // An eager step rewrites the whole state: the value-tiled kernel, which keeps
-    // its tile in registers between the read and the write, measured faster.
-    if (eager) return false;
+    // A step that rewrites every head (eager, or merging every slot) goes to the
+    // value-tiled kernel, which keeps its tile in registers between the read and
+    // the write and measured faster for it.
+    if (rewrites_all) return false;
     return (long long)a->batch * d.n_heads >= (long long)dl::device_sm_count();
 }
 
@@ -120,7 +121,7 @@ dl_status check_step(const dl_pool *P, int32_t layer, const dl_step_args *a, boo
 }
 
 dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_out,
-                   bool auto_merge, bool eager, void *stream) {
+                   int32_t auto_merge, bool eager, void *stream) {
     const dl_pool_desc &d = P->d;
     dl::KParams p = base_params(d, layer);
     p.slots = a->slots;
@@ -133,11 +134,13 @@ dl_status run_step(dl_pool *P, int32_t layer, const dl_step_args *a, bool want_o
     p.beta = d.update == DL_UPDATE_ADD ? nullptr : a->beta;
     p.out = want_out ? a->out : nullptr;
     p.auto_merge = auto_merge ? 1 : 0;
+    p.merge_every = (!eager && auto_merge == DL_MERGE_ADAPTIVE &&
+                     dl::adaptive_merges_every_step(a->batch, d.n_heads)) ? 1 : 0;
     p.eager = eager ? 1 : 0;
     p.want_out = want_out ? 1 : 0;
     p.undecayed = d.update == DL_UPDATE_DELTA_UNDECAYED ? 1 : 0;
     cudaError_t e;
-    if (use_whole_head(d, a, want_out, eager)) {
+    if (use_whole_head(d, a, want_out, eager || p.merge_every)) {
         p.nv = 1;
         e = dl::launch_whole_head(p, d.decay, d.update != DL_UPDATE_ADD, a->in_dtype == DL_BF16,
                                   static_cast<cudaStream_t>(stream));
@@ -212,21 +215,21 @@ DL_API dl_status dl_decode_step(dl_pool *pool, int32_t layer, const dl_step_args
     const dl_status s = check_step(pool, layer, args, true, true);
     if (s != DL_OK || args->batch == 0) return s;
     if (!pool->d.log) return DL_ERR_UNSUPPORTED;
-    return run_step(pool, layer, args, true, auto_merge != 0, false, stream);
+    return run_step(pool, layer, args, true, auto_merge, false, stream);
 }
 
 DL_API dl_status dl_append(dl_pool *pool, int32_t layer, const dl_step_args *args, void *stream) {
     const dl_status s = check_step(pool, layer, args, false, true);
     if (s != DL_OK || args->batch == 0) return s;
     if (!pool->d.log) return DL_ERR_UNSUPPORTED;
-    return run_step(pool, layer, args, false, false, false, stream);
+    return run_step(pool, layer, args, false, DL_MERGE_NONE, false, stream);
 }
 
 DL_API dl_status dl_eager_step(dl_pool *pool, int32_t layer, const dl_step_args *args,
                                void *stream) {
     const dl_status s = check_step(pool, layer, args, true, false);
     if (s != DL_OK || args->batch == 0) return s;
-    return run_step(pool, layer, args, true, false, true, stream);
+    return run_step(pool, layer, args, true, DL_MERGE_NONE, true, stream);
 }
 
 static dl_status merge_like(dl_pool *pool, int32_t layer, const int32_t *slots, int32_t batch,
@@ -292,6 +295,14 @@ DL_API dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void
     return host ? DL_ERR_DEVICE : DL_OK;
 }
 
+DL_API dl_status dl_merge_policy(int32_t batch, int32_t n_heads, int32_t auto_merge,
+                                 int32_t *merges_every_step) {
+    if (!merges_every_step || batch < 0 || n_heads <= 0) return DL_ERR_INVALID_ARG;
+    *merges_every_step = (auto_merge == DL_MERGE_ADAPTIVE && batch > 0 &&
+                          dl::adaptive_merges_every_step(batch, n_heads)) ? 1 : 0;
+    return DL_OK;
+}
+
 DL_API dl_status dl_debug_wait_limit(int64_t limit_ns) {
     g_wait_ns.store(limit_ns > 0 ? (unsigned long long)limit_ns : kDefaultWaitNs);
     return DL_OK;
@@ -313,6 +324,17 @@ DL_API const char *dl_status_string(dl_status status) {
 namespace dl {
 
 unsigned long long wait_limit_ns() { return g_wait_ns.load(); }
+
+// A decode launch with fewer than this many heads per SM is latency-bound: its time
+// is the dependent chain of one head (slot id, live length, log, tile) and, when a
+// slot merges, that head's write-back, not the bytes.  Measured on B200 (RetNet,
+// L = 32): 3.5 heads per SM ran faster merging every step (the eager recurrence),
+// 14 heads per SM faster deferred.
+constexpr int kAdaptiveHeadsPerSm = 6;
+
+bool adaptive_merges_every_step(long long batch, int n_heads) {
+    return batch * (long long)n_heads < (long long)kAdaptiveHeadsPerSm * device_sm_count();
+}
 
 // Checks a bare descriptor with the rules of dl_create_pool, except that its
 // arrival-counter buffer is not looked at (the entry point that allocates nothing

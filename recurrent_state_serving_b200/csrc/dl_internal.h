@@ -38,6 +38,7 @@ struct KParams {
     float *dense_out;
     // behaviour
     int auto_merge;  // decode step: the slot's merge step writes the materialised state
+    int merge_every; // decode step with auto_merge: every slot merges on every step
     int eager;       // eager step: c = 0 and always write back, no log
     int want_out;    // write o_t
     int undecayed;   // delta correction from S_{t-1} instead of Diag(e^lambda) S_{t-1}
@@ -47,6 +48,10 @@ struct KParams {
 // Bound of the kernels' pipeline waits (ns) for launches issued now: 100 ms unless
 // a test shortened it with dl_debug_wait_limit.
 unsigned long long wait_limit_ns();
+
+// Does a dl_decode_step of `batch` slots x `n_heads` heads under DL_MERGE_ADAPTIVE
+// merge every slot on every step (a launch too small to fill the GPU)?
+bool adaptive_merges_every_step(long long batch, int n_heads);
 
 // Value-tile width chosen for a launch (16 or 32 columns).
 int pick_bv(int dk, int dv, long long work_items_at_32);

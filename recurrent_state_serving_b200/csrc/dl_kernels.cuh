@@ -107,7 +107,7 @@ struct DynLayout {
 //   y_q = Sbar^T qt + sum_i cq_i b_i,  y_k = Sbar^T kt + sum_i ck_i b_i
 //   b_t = v (additive) | beta (v - y_k) (delta);  o_t = y_q + b_t (k . q)
 // then either append (k, b_t, lbar_t) as entry c, or, on the slot's merge step
-// (and always in eager mode), write
+// (on every step with p.merge_every, and always in eager mode), write
 //   S_t = e^{lbar_t} (.) Sbar + sum_i A'_i b_i^T + k b_t^T,  A'_i = a_i (.) e^{lbar_t - Lambda_i}.
 // ---------------------------------------------------------------------------
 template <int DK, int BV, int DECAY, bool DELTA, typename IT>
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         leave();
         return;
     }
-    const bool merge_now = p.eager || (p.auto_merge && c >= p.L - 1);
+    const bool merge_now = p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every));
     if (!merge_now && c >= p.L) {
         if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_FULL);
         leave();

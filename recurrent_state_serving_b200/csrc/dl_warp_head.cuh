@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     // with no more heads than warps every warp has one head and the order is moot
     const bool pre = kc > NW && kc <= KMAX;
     auto merges = [&](int s, int c) {
-        return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && c >= p.L - 1));
+        return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every)));
     };
     // Merges written during pass 1 (no delta rule, at most TM_ENT entries) split in two
     // when the CTA has few heads: a merge head costs about three append heads, so with
@@ -325,11 +325,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             if (c != 0) hd.st = DL_EBIT_LIVE_LOG;
         } else if (c < 0 || c > p.L) {
             hd.st = DL_EBIT_LOG_LEN;
-        } else if (!(p.auto_merge && c >= p.L - 1) && c >= p.L) {
+        } else if (!(p.auto_merge && (c >= p.L - 1 || p.merge_every)) && c >= p.L) {
             hd.st = DL_EBIT_LOG_FULL;
         }
         if (hd.st) return;
-        const bool merge = p.eager || (p.auto_merge && c >= p.L - 1);
+        const bool merge = p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every));
         hd.mk = !merge ? MK_APPEND : c > TM_ENT ? MK_ROUNDS : DELTA ? MK_PASS2 : MK_FUSED;
         hd.nl = (c + EPC - 1) / EPC;
         hd.n = hd.nl + (hd.half ? NCH / 2 : NCH) + (hd.mk == MK_PASS2 ? NCH : 0);

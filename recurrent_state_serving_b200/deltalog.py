@@ -33,6 +33,16 @@ LOG_FORMAT = {"fp32": 0, "compact": 1}
 REPLAY = {"per_tile": 0, "cluster": 1}
 DL_EBIT_SLOT_RANGE, DL_EBIT_LOG_FULL, DL_EBIT_LIVE_LOG, DL_EBIT_LOG_LEN, DL_EBIT_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
+DL_MERGE_NONE, DL_MERGE_AT_CAPACITY, DL_MERGE_ADAPTIVE = 0, 1, 2
+MERGE = {False: DL_MERGE_NONE, True: DL_MERGE_AT_CAPACITY, "none": DL_MERGE_NONE,
+         "capacity": DL_MERGE_AT_CAPACITY, "adaptive": DL_MERGE_ADAPTIVE}
+
+
+def merge_code(auto_merge) -> int:
+    """auto_merge as the C ABI's int: a bool, 'none' / 'capacity' / 'adaptive', or a DL_MERGE_* value."""
+    if isinstance(auto_merge, (bool, str)):
+        return MERGE[auto_merge]
+    return int(auto_merge)
 
 
 class dl_pool_desc(ctypes.Structure):
@@ -68,11 +78,12 @@ _lib.dl_read_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), ctypes.c_int
 _lib.dl_decode_step_noalloc.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.c_int32,
                                         ctypes.POINTER(dl_step_args), ctypes.c_int32, _vp]
 _lib.dl_debug_wait_limit.argtypes = [ctypes.c_int64]
+_lib.dl_merge_policy.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
 _lib.dl_status_string.argtypes = [ctypes.c_int]
 _lib.dl_status_string.restype = ctypes.c_char_p
 for _f in ("dl_log_bytes", "dl_create_pool", "dl_destroy_pool", "dl_decode_step", "dl_append", "dl_eager_step",
            "dl_merge", "dl_materialize", "dl_reset_slots", "dl_read_error", "dl_decode_step_noalloc",
-           "dl_debug_wait_limit"):
+           "dl_debug_wait_limit", "dl_merge_policy"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -208,7 +219,7 @@ def dl_decode_step(pool: Pool, layer: int, slots, q, k, v, lam=None, beta=None, 
         out = torch.empty(slots.numel(), pool.n_heads, pool.d_v, dtype=torch.float32,
                           device=pool.state.device)
     a = _step_args(pool, slots, q, k, v, lam, beta, out, lambda_per_head)
-    _check(_lib.dl_decode_step(pool.handle, layer, ctypes.byref(a), 1 if auto_merge else 0,
+    _check(_lib.dl_decode_step(pool.handle, layer, ctypes.byref(a), merge_code(auto_merge),
                                _stream(stream)), "dl_decode_step")
     return out
 
@@ -227,7 +238,7 @@ def dl_decode_step_noalloc(pool: Pool, layer: int, slots, q, k, v, lam=None, bet
     desc = dl_pool_desc.from_buffer_copy(pool.desc)
     desc.arrive = None
     _check(_lib.dl_decode_step_noalloc(ctypes.byref(desc), layer, ctypes.byref(a),
-                                       1 if auto_merge else 0, _stream(stream)),
+                                       merge_code(auto_merge), _stream(stream)),
            "dl_decode_step_noalloc")
     return out
 
@@ -284,6 +295,14 @@ def dl_read_error(pool: Pool, clear=True, stream=None) -> int:
     return int(bits.value)
 
 
+def dl_merge_policy(batch: int, n_heads: int, auto_merge="adaptive") -> bool:
+    """Whether dl_decode_step of this batch merges every slot on every step."""
+    out = ctypes.c_int32(0)
+    _check(_lib.dl_merge_policy(int(batch), int(n_heads), merge_code(auto_merge), ctypes.byref(out)),
+           "dl_merge_policy")
+    return bool(out.value)
+
+
 def dl_debug_wait_limit(limit_ns: int = 0):
     """Test hook: bound of the whole-head kernel's pipeline waits for later launches
     (process-wide); limit_ns <= 0 restores the default 100 ms."""
@@ -311,7 +330,7 @@ class PreparedStep:
         self.args = _step_args(pool, slots, q, k, v, lam, beta, None if kind == "append" else out,
                                lambda_per_head)
         self._ref = ctypes.byref(self.args)
-        self._auto = 1 if auto_merge else 0
+        self._auto = merge_code(auto_merge)
 
     def __call__(self, stream=None) -> int:
         st = _stream(stream)

@@ -38,11 +38,12 @@ class DecodeRunner:
     def __init__(self, wl: synth.Workload, *, n_slots: int | None = None, slot_seed: int | None = None,
                  layers=None, mode: str = "deferred", update: str | None = None,
                  device: str = "cuda", tile_v: int = 0, n_groups: int = 1, log_format: str = "fp32",
-                 replay: str = "per_tile", offsets=None):
+                 replay: str = "per_tile", offsets=None, merge="capacity"):
         if mode not in ("deferred", "eager"):
             raise ValueError(mode)
         self.wl = wl
         self.mode = mode
+        self.merge = merge   # dl_decode_step's merge policy: 'capacity', 'adaptive' or 'none'
         self.update = update or wl.update
         self.device = torch.device(device)
         self.layers = list(range(wl.n_layers)) if layers is None else list(layers)
@@ -111,9 +112,13 @@ class DecodeRunner:
     def call(self, layer: int, x: dict, slots=None, out=None, stream=None):
         """One library call for one layer (decode step or eager step)."""
         slots = self.slots if slots is None else slots
-        fn = dl.dl_decode_step if self.mode == "deferred" else dl.dl_eager_step
-        return fn(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"],
-                  out=out, lambda_per_head=self.wl.lambda_const, stream=stream)
+        if self.mode == "eager":
+            return dl.dl_eager_step(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"],
+                                    beta=x["beta"], out=out, lambda_per_head=self.wl.lambda_const,
+                                    stream=stream)
+        return dl.dl_decode_step(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"],
+                                 beta=x["beta"], out=out, lambda_per_head=self.wl.lambda_const,
+                                 auto_merge=self.merge, stream=stream)
 
     def run_presteps(self, inputs=None):
         """Staggering: slot b of group g takes group_offsets[g, b] untimed decode steps

@@ -10,7 +10,7 @@ import torch
 from recurrent_state_serving_b200 import deltalog as dl
 
 EXPECTED = ["dl_append", "dl_create_pool", "dl_debug_wait_limit", "dl_decode_step", "dl_decode_step_noalloc",
-            "dl_destroy_pool", "dl_eager_step", "dl_log_bytes", "dl_materialize", "dl_merge",
+            "dl_destroy_pool", "dl_eager_step", "dl_log_bytes", "dl_materialize", "dl_merge", "dl_merge_policy",
             "dl_read_error", "dl_reset_slots", "dl_status_string"]
 
 
@@ -282,3 +282,19 @@ def test_header_compiles_as_c99_and_matches_the_binding(tmp_path):
             n += 1
     assert n == 22
     assert run.stdout.strip().endswith("OK")
+
+
+def test_merge_policy_without_gpu():
+    """DL_MERGE_ADAPTIVE merges every step only below a few heads per SM (148 SMs
+    assumed when no device is visible); other policies never do."""
+    assert dl.dl_merge_policy(1, 32, "adaptive")            # 32 heads
+    assert dl.dl_merge_policy(16, 32, "adaptive")           # 512 heads
+    assert not dl.dl_merge_policy(64, 32, "adaptive")       # 2048 heads
+    assert not dl.dl_merge_policy(256, 32, "adaptive")
+    assert not dl.dl_merge_policy(1, 32, "capacity") and not dl.dl_merge_policy(1, 32, False)
+    assert not dl.dl_merge_policy(0, 32, "adaptive")
+    out = ctypes.c_int32(5)
+    assert dl.library().dl_merge_policy(1, 0, 2, ctypes.byref(out)) == dl.DL_ERR_INVALID_ARG
+    assert dl.library().dl_merge_policy(-1, 4, 2, ctypes.byref(out)) == dl.DL_ERR_INVALID_ARG
+    assert dl.library().dl_merge_policy(1, 4, 2, None) == dl.DL_ERR_INVALID_ARG
+    assert dl.merge_code(True) == 1 and dl.merge_code("adaptive") == 2 and dl.merge_code(0) == 0

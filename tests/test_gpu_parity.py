@@ -463,3 +463,47 @@ def test_read_error_clears_only_when_asked():
     assert dl.dl_read_error(r.pool, clear=False) == dl.DL_EBIT_SLOT_RANGE
     assert dl.dl_read_error(r.pool, clear=True) == dl.DL_EBIT_SLOT_RANGE
     assert dl.dl_read_error(r.pool, clear=False) == 0
+
+
+@pytest.mark.parametrize("name", ["gdn_gva", "retnet", "kda"])
+def test_adaptive_policy_matches_the_oracle(name):
+    """DL_MERGE_ADAPTIVE on launches below a few heads per SM merges every slot on every
+    step; switched on mid-run it first folds the live logs.  Outputs and states match
+    the oracle under either policy, and the log stays empty once adaptive."""
+    wl = REDUCED[name]
+    assert dl.dl_merge_policy(wl.batch, wl.n_heads, "adaptive")
+    T = 40
+    half = 13
+    r = DecodeRunner(wl, n_slots=wl.batch + 2, slot_seed=4, tile_v=0)
+    r.load_initial_state()
+    r.run_presteps()
+    outs = {l: [] for l in r.layers}
+    ck = {l: [] for l in r.layers}
+    for t in range(T):
+        r.merge = "capacity" if t < half else "adaptive"
+        for l in r.layers:
+            outs[l].append(r.call(l, r.gen_inputs(t, l)).double().cpu().numpy())
+            if t + 1 in (half, T):
+                ck[l].append(r.materialize(l).double().cpu().numpy())
+        if t >= half:
+            assert int(r.pool.log_len.abs().sum()) == 0
+    assert r.errors() == 0
+    for l in r.layers:
+        O, S = H.oracle_reference(wl, l, T, ckpts=[half, T])
+        H.check_steps(np.stack(outs[l]), O, what=f"{name} layer {l} output")
+        H.check_steps(np.stack(ck[l]), S, elem=None, what=f"{name} layer {l} state")
+
+
+def test_adaptive_policy_is_capacity_on_large_launches():
+    """Above the threshold the adaptive policy is the at-capacity one: same outputs,
+    same logs, bit for bit."""
+    wl = synth.GLA_DIAG.with_(batch=64, n_heads=16, n_kheads=16, steps=12, log_cap=4)
+    assert not dl.dl_merge_policy(wl.batch, wl.n_heads, "adaptive")
+    res = []
+    for merge in ("capacity", "adaptive"):
+        r = DecodeRunner(wl, merge=merge)
+        o, _, _ = H.gpu_rollout(r, wl.steps)
+        res.append((o[0], r.pool.log.clone(), r.pool.log_len.clone(), r.pool.state.clone()))
+    np.testing.assert_array_equal(res[0][0], res[1][0])
+    for a, b in zip(res[0][1:], res[1][1:]):
+        assert torch.equal(a, b)
