@@ -94,6 +94,8 @@ def parse(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--log-cap", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's layer count (small cases for profiling)")
     ap.add_argument("--subs", default=DEFAULT_SUBS,
                     help="comma list of name[:bB][:LL] sub-records, or 'none'")
     ap.add_argument("--merge-legs", default=DEFAULT_MERGE_LEGS,
@@ -126,7 +128,7 @@ def parse(argv=None):
 
 
 def parse_spec(spec: str):
-    """'name[:bB][:LL]' -> a synth workload with that batch / log capacity."""
+    """'name[:bB][:LL][:nN]' -> a synth workload with that batch / log capacity / layer count."""
     from recurrent_state_serving_b200 import synth
     parts = spec.strip().split(":")
     if parts[0] not in synth.WORKLOADS:
@@ -137,6 +139,8 @@ def parse_spec(spec: str):
             wl = wl.with_(batch=int(p[1:]))
         elif p.startswith("L"):
             wl = wl.with_(log_cap=int(p[1:]))
+        elif p.startswith("n"):
+            wl = wl.with_(n_layers=int(p[1:]))
         else:
             raise SystemExit(f"bad workload spec {spec!r}")
     return wl
@@ -154,6 +158,8 @@ def workload(a):
         wl = wl.with_(log_cap=a.log_cap)
     if a.batch:
         wl = wl.with_(batch=a.batch)
+    if a.layers:
+        wl = wl.with_(n_layers=a.layers)
     return wl
 
 

@@ -282,16 +282,17 @@ dl_status dl_materialize(dl_pool *pool, int32_t layer, const int32_t *slots, int
  * arrival counters part-way through the step. */
 dl_status dl_read_error(dl_pool *pool, int32_t *bits, int32_t clear, void *stream);
 
-/* Fault injection for tests (the paper has no counterpart).  Sets, process-wide,
- * the time limit of the whole-head decode kernel's pipeline waits (a bulk copy's
- * arrival, a split merge head's partial output) for launches issued after the
- * call; limit_ns <= 0 restores the default of 100 ms.  A short limit makes waits
- * run out: the kernel then sets DL_EBIT_TIMEOUT, stops the affected work, waits
- * with the default 100 ms bound for its own bulk copies still in flight, frees its
- * tensor memory and returns, so the context stays usable.  The slots of such a
- * call must then be prefilled and reset (see dl_read_error).  Always DL_OK; makes
- * no CUDA call. */
-dl_status dl_debug_wait_limit(int64_t limit_ns);
+/* Fault injection for tests (the paper has no counterpart).  While limit_ns > 0
+ * (process-wide, for launches issued after the call), every launch of the
+ * whole-head decode kernel makes the first warp of its first CTA wait, bounded by
+ * limit_ns, on a barrier that nothing completes, before that warp consumes any of
+ * the bulk copies it has already issued.  The wait runs out: the kernel sets
+ * DL_EBIT_TIMEOUT, the warp stops, waits with the normal 100 ms bound for its own
+ * copies still in flight, the CTA frees its tensor memory and returns, and the
+ * context stays usable.  The heads of that warp are left unprocessed, so the
+ * call's slots must be prefilled and reset afterwards (see dl_read_error).
+ * limit_ns <= 0 switches it off.  Always DL_OK; makes no CUDA call. */
+dl_status dl_debug_stall(int64_t limit_ns);
 
 /* Decode step that allocates nothing.  The paper has no counterpart: this entry
  * point exists for integration only.

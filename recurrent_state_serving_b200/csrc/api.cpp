@@ -19,8 +19,7 @@ struct dl_pool {
 
 namespace {
 
-constexpr unsigned long long kDefaultWaitNs = 100000000ull;  // 100 ms
-std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+std::atomic<unsigned long long> g_stall_ns{0};
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -70,7 +69,7 @@ dl::KParams base_params(const dl_pool_desc &d, int layer) {
     p.b16 = l.b16;
     p.layer = layer;
     p.cl = 1;
-    p.wait_ns = dl::wait_limit_ns();
+    p.stall_ns = dl::stall_ns();
     return p;
 }
 
@@ -246,10 +245,14 @@ static dl_status merge_like(dl_pool *pool, int32_t layer, const int32_t *slots, 
     p.slots = slots;
     p.batch = batch;
     p.dense_out = dense_out;
-    int bv = 32;
-    set_tiles(d, p, batch, bv);
-    const cudaError_t e = dl::launch_merge(p, bv, d.decay, materialize,
-                                           static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (dl::whole_head_supported(d.d_k, d.d_v) && d.tile_v != 16 && d.tile_v != 32) {
+        e = dl::launch_merge_head(p, d.decay, materialize, static_cast<cudaStream_t>(stream));
+    } else {
+        int bv = 32;
+        set_tiles(d, p, batch, bv);
+        e = dl::launch_merge(p, bv, d.decay, materialize, static_cast<cudaStream_t>(stream));
+    }
     return e == cudaSuccess ? DL_OK : DL_ERR_CUDA;
 }
 
@@ -303,8 +306,8 @@ DL_API dl_status dl_merge_policy(int32_t batch, int32_t n_heads, int32_t auto_me
     return DL_OK;
 }
 
-DL_API dl_status dl_debug_wait_limit(int64_t limit_ns) {
-    g_wait_ns.store(limit_ns > 0 ? (unsigned long long)limit_ns : kDefaultWaitNs);
+DL_API dl_status dl_debug_stall(int64_t limit_ns) {
+    g_stall_ns.store(limit_ns > 0 ? (unsigned long long)limit_ns : 0ull);
     return DL_OK;
 }
 
@@ -323,7 +326,7 @@ DL_API const char *dl_status_string(dl_status status) {
 
 namespace dl {
 
-unsigned long long wait_limit_ns() { return g_wait_ns.load(); }
+unsigned long long stall_ns() { return g_stall_ns.load(); }
 
 // A decode launch with fewer than this many heads per SM is latency-bound: its time
 // is the dependent chain of one head (slot id, live length, log, tile) and, when a

@@ -42,12 +42,11 @@ struct KParams {
     int eager;       // eager step: c = 0 and always write back, no log
     int want_out;    // write o_t
     int undecayed;   // delta correction from S_{t-1} instead of Diag(e^lambda) S_{t-1}
-    unsigned long long wait_ns;  // bound on the whole-head kernel's pipeline waits
+    unsigned long long stall_ns;  // timeout test: 0, or the bound of a wait that never completes
 };
 
-// Bound of the kernels' pipeline waits (ns) for launches issued now: 100 ms unless
-// a test shortened it with dl_debug_wait_limit.
-unsigned long long wait_limit_ns();
+// dl_debug_stall's setting for launches issued now (0: off).
+unsigned long long stall_ns();
 
 // Does a dl_decode_step of `batch` slots x `n_heads` heads under DL_MERGE_ADAPTIVE
 // merge every slot on every step (a launch too small to fill the GPU)?
@@ -65,6 +64,8 @@ cudaError_t launch_whole_head(const KParams &p, int decay, bool delta, bool bf16
 
 cudaError_t launch_merge(const KParams &p, int bv, int decay, bool materialize,
                          cudaStream_t st);
+// Merge / materialise of whole 128 x 128 heads, one CTA per head.
+cudaError_t launch_merge_head(const KParams &p, int decay, bool materialize, cudaStream_t st);
 cudaError_t launch_reset(const int32_t *slots, int batch, int n_slots, int n_layers,
                          int32_t *log_len, int32_t *arrive, int32_t *err, cudaStream_t st);
 // Atomically clears `bits` in the error word (bits set meanwhile by other launches survive).

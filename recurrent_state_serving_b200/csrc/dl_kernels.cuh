@@ -405,8 +405,10 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
             __stcs(reinterpret_cast<float4 *>(tile + (size_t)(rg + m * RG) * dv) + quad, Sr[m]);
     }
 
-    // 8. Finalize: the last CTA of this (slot, layer) commits the live length
-    if (!p.eager) {
+    // 8. Finalize: the last CTA of this (slot, layer) commits the live length.  A merge
+    //    step that started from an empty log leaves it empty: nothing to commit, and
+    //    every CTA of the slot saw the same c, so none of them counts itself in.
+    if (!p.eager && !(merge_now && c == 0)) {
         __syncthreads();
         if (tid == 0) {
             __threadfence();
@@ -515,6 +517,134 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
             __threadfence();
             const int old = atomicAdd(p.arrive + sl, 1);
             if (old == p.H * nv - 1) {
+                p.log_len[sl] = 0;
+                p.arrive[sl] = 0;
+            }
+        }
+    }
+}
+
+}  // namespace dl
+
+namespace dl {
+
+// ---------------------------------------------------------------------------
+// Merge / materialise of whole 128 x 128 heads (DeltaLog paper, Section 3.3,
+// Merge: each dense fp32 tile is rewritten once).  One CTA of eight warps owns a
+// (slot, head): warp w holds rows 16w .. 16w+15 of the tile in registers (lane l
+// columns 4l .. 4l+3), loaded with streaming 128-bit loads before anything else is
+// read.  The CTA forms A'^T[i][r] = a_i[r] e^{lbar[r] - Lambda_i[r]} and b_i for
+// the c live entries once, in shared memory; every lane then applies
+//   Sbar'[r][:] = e^{lbar[r]} Sbar[r][:] + sum_i A'^T[i][r] b_i[:]
+// to its 16 rows, reading b_i (its four columns) and A'^T[i][16w..16w+15]
+// (broadcast) from shared memory.  Merge writes Sbar' over the base and commits
+// live length 0 (the last CTA of the slot); materialise writes it to dense_out.
+// ---------------------------------------------------------------------------
+constexpr int MH_NT = 256;
+
+template <int DECAY>
+__global__ void __launch_bounds__(MH_NT, 2) merge_head_kernel(const KParams p, const int materialize)
+{
+    constexpr int D = 128, RW = 16;
+    extern __shared__ __align__(16) float s_dyn[];
+    __shared__ __align__(16) float s_e[D];
+    __shared__ __align__(16) float s_lb[D];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int bi = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int s = p.slots[bi];
+    if (s < 0 || s >= p.n_slots) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_SLOT_RANGE);
+        return;
+    }
+    const size_t sl = (size_t)s * p.n_layers + p.layer;
+    const size_t head = sl * p.H + h;
+    float *tile = p.state + head * (size_t)(D * D);
+    const int c = p.log_len[sl];
+    if (c < 0 || c > p.L) {
+        if (tid == 0) atomicOr(p.err, DL_EBIT_LOG_LEN);
+        return;
+    }
+    if (!materialize && c == 0) return;  // nothing to fold; live length stays 0
+
+    // 1. the tile rows of this warp, in flight while the log is read
+    float4 S[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+        S[r] = __ldcs(reinterpret_cast<const float4 *>(tile + (size_t)(RW * w + r) * D) + lane);
+
+    // 2. lbar = Lambda_{c-1}, e^{lbar}; A'^T and b of the live entries
+    const float *ring = p.log + head * (size_t)p.L * p.E;
+    float *sA = s_dyn;                        // [c][D]  A'^T
+    float *sB = s_dyn + (size_t)p.L * D;      // [c][D]  b
+    for (int r = tid; r < D; r += MH_NT) {
+        float lb = 0.f;
+        if (c > 0 && DECAY == DL_DECAY_DIAG) lb = ring[(size_t)(c - 1) * p.E + p.loff + r];
+        if (c > 0 && DECAY == DL_DECAY_SCALAR) lb = ring[(size_t)(c - 1) * p.E + p.loff];
+        s_lb[r] = lb;
+        s_e[r] = DECAY == DL_DECAY_NONE ? 1.f : expf(lb);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < c * (D / 4); idx += MH_NT) {
+        const int i = idx / (D / 4), r4 = idx % (D / 4);
+        const float *ent = ring + (size_t)i * p.E;
+        float4 a4 = ent_a4(p, ent, r4);
+        if (DECAY == DL_DECAY_DIAG) {
+            const float4 L4 = *reinterpret_cast<const float4 *>(ent + p.loff + 4 * r4);
+            const float4 lb4 = reinterpret_cast<const float4 *>(s_lb)[r4];
+            a4.x *= expf(lb4.x - L4.x);
+            a4.y *= expf(lb4.y - L4.y);
+            a4.z *= expf(lb4.z - L4.z);
+            a4.w *= expf(lb4.w - L4.w);
+        } else if (DECAY == DL_DECAY_SCALAR) {
+            const float g = expf(s_lb[0] - ent[p.loff]);
+            a4.x *= g;
+            a4.y *= g;
+            a4.z *= g;
+            a4.w *= g;
+        }
+        reinterpret_cast<float4 *>(sA + (size_t)i * D)[r4] = a4;
+        reinterpret_cast<float4 *>(sB + (size_t)i * D)[r4] = ent_b4(p, ent, r4);
+    }
+    __syncthreads();
+
+    // 3. the rank-c update of this warp's rows
+#pragma unroll
+    for (int r4 = 0; r4 < RW / 4; ++r4) {
+        const float4 e4 = reinterpret_cast<const float4 *>(s_e + RW * w)[r4];
+        const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            float4 &v = S[4 * r4 + y];
+            v.x *= ev[y];
+            v.y *= ev[y];
+            v.z *= ev[y];
+            v.w *= ev[y];
+        }
+    }
+    for (int i = 0; i < c; ++i) {
+        const float4 b4 = reinterpret_cast<const float4 *>(sB + (size_t)i * D)[lane];
+        const float4 *arow = reinterpret_cast<const float4 *>(sA + (size_t)i * D + RW * w);
+#pragma unroll
+        for (int r4 = 0; r4 < RW / 4; ++r4) {
+            const float4 a4 = arow[r4];
+            fma4(S[4 * r4 + 0], a4.x, b4);
+            fma4(S[4 * r4 + 1], a4.y, b4);
+            fma4(S[4 * r4 + 2], a4.z, b4);
+            fma4(S[4 * r4 + 3], a4.w, b4);
+        }
+    }
+    float *dst = materialize ? p.dense_out + ((size_t)bi * p.H + h) * (size_t)(D * D) : tile;
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+        __stcs(reinterpret_cast<float4 *>(dst + (size_t)(RW * w + r) * D) + lane, S[r]);
+
+    // 4. Finalize (merge): the last CTA of this (slot, layer) commits live length 0
+    if (!materialize) {
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const int old = atomicAdd(p.arrive + sl, 1);
+            if (old == p.H - 1) {
                 p.log_len[sl] = 0;
                 p.arrive[sl] = 0;
             }

@@ -41,11 +41,12 @@
 // of them than warps (and at most KMAX), the CTA first reads every head's slot id and
 // live length (all threads at once) and puts the merge steps first: a merge head
 // costs several append heads, and started early it overlaps their streaming instead
-// of ending the launch alone.  A merge without the delta rule is split in two work
-// items, each streaming and rewriting half of the tile's rows (both stage the
-// coefficients in their own TMEM share); the second to finish adds the first's partial
-// output (left in `out`) to its own and commits the head.  Warps take the items in
-// that order from a shared counter.
+// of ending the launch alone.  When the CTA has few heads, a merge without the delta
+// rule is split into 2 or 4 work items, each streaming and rewriting its share of the
+// tile's rows (each stages the coefficients in its own TMEM share) and adding its
+// partial output into a shared-memory accumulator of the head; the last part to
+// arrive adds the token term, writes o_t and commits the head.  Nothing waits for
+// another part.  Warps take the items in that order from a shared counter.
 //
 // The kernel is instantiated per log layout (FMT 0: fp32 rows; FMT 1: compact rows,
 // bf16 a_i and, without the delta rule, bf16 b_i), which fixes how many entries a
@@ -53,10 +54,11 @@
 // programmatic stream serialization: a CTA sets up its mbarriers and TMEM while the
 // previous kernel in the stream finishes, and reads global memory only after it.
 //
-// Every wait is bounded (p.wait_ns, 100 ms unless a test shortens it); a warp whose
-// wait runs out sets DL_EBIT_TIMEOUT, stops, and waits (bounded by the fixed 100 ms
-// WAIT_NS, whatever p.wait_ns is) for its own copies still in flight before the
-// CTA frees its tensor memory and exits.
+// Every wait is bounded (100 ms); a warp whose wait runs out sets DL_EBIT_TIMEOUT,
+// stops, and waits (bounded again) for its own copies still in flight before the
+// CTA frees its tensor memory and exits.  A test can make that happen on purpose
+// (p.stall_ns): the first warp of the first CTA then waits, bounded by stall_ns, on
+// a barrier that nothing completes, before it consumes anything of its stream.
 #pragma once
 
 #include "dl_kernels.cuh"
@@ -75,8 +77,8 @@ constexpr int NTHREADS = NW * 32;
 constexpr int NSW = 3;                      // stages per warp
 constexpr int RPB = 4;                      // log entries per load block (merge rounds)
 constexpr int MRB = CF / (DK + DV);         // entries per merge round (A' and b in one stage)
-constexpr uint64_t WAIT_NS = 100000000ull;  // bound on the abort path's drain waits
-constexpr int NB = NSW + 2;                 // mbarriers per warp: stream stages + merge re-stream
+constexpr uint64_t WAIT_NS = 100000000ull;  // bound on every wait
+constexpr int NB = NSW + 3;                 // mbarriers per warp: stream stages, merge re-stream, stall test
 constexpr int TM_ENT = 32;                  // merge entries staged in TMEM per warp
 constexpr uint32_t TM_COLS = 512;           // TMEM columns per CTA (all of them)
 constexpr uint32_t TM_WCOLS = 256;          // per warp: two warps share each lane quarter
@@ -84,11 +86,15 @@ constexpr int AG = 4;                       // merge entries per TMEM load / sha
 // per-warp scratch: the head's row vectors qt, kt, e^{lbar_t}, k, lbar_t (5 x 128 floats)
 // and the A' values of AG entries for the 16 rows of one block
 constexpr int WSCR = 5 * DK + AG * CR;
-// per-CTA head list: slot id, live length, halves' combine state of up to KMAX heads,
-// and the processing order (a split merge head takes two positions)
+// per-CTA head list: slot id, live length, split combine state of up to KMAX heads,
+// and the processing order (a head split in S parts takes S positions)
 constexpr int KMAX = 512;
+constexpr int MAX_PARTS = 4;                // parts of a split merge head
+constexpr int NPA = 8;                      // split heads in flight per CTA (accumulators)
 constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4 + (size_t)NW * NB * 8 + 32 +
-                        (size_t)KMAX * (4 + 4 + 4) + (size_t)2 * KMAX * 2;
+                        (size_t)KMAX * (4 + 4 + 4) + (size_t)2 * KMAX * 2 + (size_t)NPA * DV * 4;
+static_assert(KMAX + (MAX_PARTS - 1) * NPA <= 2 * KMAX, "the order holds every head and every extra part");
+static_assert(SMEM <= 232448, "a CTA may use at most 227 KB of shared memory");
 static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
 static_assert(TM_ENT * 8 <= (int)TM_WCOLS, "A'_i and b_i take 8 columns per entry");
 constexpr unsigned FULL = 0xffffffffu;
@@ -148,7 +154,8 @@ struct Head {
     int mk;        // MergeKind
     int nl;        // log chunks in its stream
     int n;         // stream positions: nl + NCH (+ NCH for MK_PASS2); 0 when skipped
-    int half;      // 0: the whole head; 1 / 2: rows 0..63 / 64..127 of a split merge
+    int part;      // 0: the whole head; 1..np: rows (part-1)*128/np .. part*128/np - 1 of a split merge
+    int np;        // parts of a split merge head
     size_t head;   // (slot, layer, head) index
 };
 
@@ -194,13 +201,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     unsigned char *bars = smem + (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4;
     uint64_t *fb = reinterpret_cast<uint64_t *>(bars) + w * NB;
     uint64_t *pb = fb + NSW;  // round-wise merge: tile re-stream through stages 0 and 1
+    uint64_t *stall_bar = fb + NSW + 2;  // nothing ever arrives on it (timeout test)
     int *next_k = reinterpret_cast<int *>(bars + (size_t)NW * NB * 8);
     uint32_t *tm_slot = reinterpret_cast<uint32_t *>(next_k + 1);
-    int *cnt = next_k + 2;  // merge positions, next merge position, next other position, splits
+    int *cnt = next_k + 2;  // merge positions, next merge position, next other position, extra parts,
+                            // accumulators taken
     int *pre_slot = next_k + 8;
     int *pre_len = pre_slot + KMAX;
-    int *comb = pre_len + KMAX;  // split merge heads: halves arrived (1, 2) + 4 once a partial is in out
-    uint16_t *order = reinterpret_cast<uint16_t *>(comb + KMAX);  // k | half << 10
+    int *comb = pre_len + KMAX;  // split merge heads: (accumulator + 1) << 8 | parts arrived
+    uint16_t *order = reinterpret_cast<uint16_t *>(comb + KMAX);  // k | part << 10 | log2(parts) << 13
+    float *pacc = reinterpret_cast<float *>(order + 2 * KMAX);  // NPA x DV partial outputs
 
     // merges with live entries need tensor memory (auto-merge decode steps only)
     const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
@@ -210,8 +220,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     }
     if (threadIdx.x == 0) {
         *next_k = NW;  // warp w starts with the CTA's w-th head
-        cnt[0] = cnt[1] = cnt[2] = cnt[3] = 0;
+        cnt[0] = cnt[1] = cnt[2] = cnt[3] = cnt[4] = 0;
     }
+    for (int i = threadIdx.x; i < NPA * DV; i += NTHREADS) pacc[i] = 0.f;
     if (use_tm && w == 0) {
         ptx::tmem_alloc(tm_slot, TM_COLS);
         ptx::tmem_relinquish();
@@ -232,18 +243,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     const int n_items = p.batch * p.H;
     const int G = gridDim.x, bx = blockIdx.x;
     const int kc = bx < n_items ? (n_items - 1 - bx) / G + 1 : 0;  // heads of this CTA
-    // with no more heads than warps every warp has one head and the order is moot
-    const bool pre = kc > NW && kc <= KMAX;
+    // the head list is built when there is an order to choose (more heads than warps)
+    // or spare warps to split a merge head over
+    const bool pre = kc > 1 && kc <= KMAX;
     auto merges = [&](int s, int c) {
         return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every)));
     };
-    // Merges written during pass 1 (no delta rule, at most TM_ENT entries) split in two
-    // when the CTA has few heads: a merge head costs about three append heads, so with
-    // fewer than three heads per warp it would outlast the rest of the CTA's work; with
-    // more, the other heads hide it and a split only adds the second half's log read.
+    // Merges written during pass 1 (no delta rule, at most TM_ENT entries) are split
+    // when the CTA has few heads: a merge head costs several append heads (its
+    // write-back is a chain of c-term updates run by one warp), so with fewer than
+    // three heads per warp it would outlast the rest of the CTA's work; with more,
+    // the other heads hide it and a split only adds the parts' log reads.  Parts:
+    // with fewer heads than warps, as many as the idle warps allow (2 or 4); else 2,
+    // or 4 for logs of 16 entries or more.
     const bool split_ok = kc < 3 * NW;
-    auto splits = [&](int s, int c) {
-        return split_ok && !DELTA && !p.eager && p.want_out && merges(s, c) && c >= 0 && c <= TM_ENT;
+    auto parts_of = [&](int s, int c) -> int {
+        if (!(split_ok && !DELTA && !p.eager && p.want_out && merges(s, c) && c >= 0 && c <= TM_ENT)) return 1;
+        if (kc < NW) return NW - kc >= 3 ? 4 : NW - kc >= 1 ? 2 : 1;
+        return c >= 16 ? 4 : 2;
     };
     if (pre) {
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
@@ -251,18 +268,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             const int c = (s >= 0 && s < p.n_slots && p.log_len) ? p.log_len[(size_t)s * p.n_layers + p.layer] : 0;
             pre_slot[k] = s;
             pre_len[k] = c;
-            comb[k] = 0;
-            if (merges(s, c)) atomicAdd(&cnt[0], splits(s, c) ? 2 : 1);
-            if (splits(s, c)) atomicAdd(&cnt[3], 1);
+            int np = parts_of(s, c);
+            int cm = 0;
+            if (np > 1) {  // a split head needs one of the NPA accumulators
+                const int a = atomicAdd(&cnt[4], 1);
+                if (a < NPA) cm = (a + 1) << 8;
+                else np = 1;
+            }
+            comb[k] = cm;
+            if (merges(s, c)) atomicAdd(&cnt[0], np);
+            if (np > 1) atomicAdd(&cnt[3], np - 1);
         }
         __syncthreads();
         const int nm = cnt[0];
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
             const int s = pre_slot[k], c = pre_len[k];
-            if (splits(s, c)) {
-                const int pos = atomicAdd(&cnt[1], 2);  // the two halves next to each other
-                order[pos] = (uint16_t)(k | (1 << 10));
-                order[pos + 1] = (uint16_t)(k | (2 << 10));
+            if (comb[k] != 0) {
+                const int np = parts_of(s, c), lg = np == 4 ? 2 : 1;
+                const int pos = atomicAdd(&cnt[1], np);  // the parts next to each other
+                for (int j = 0; j < np; ++j) order[pos + j] = (uint16_t)(k | ((j + 1) << 10) | (lg << 13));
             } else {
                 const int pos = merges(s, c) ? atomicAdd(&cnt[1], 1) : nm + atomicAdd(&cnt[2], 1);
                 order[pos] = (uint16_t)k;
@@ -271,21 +295,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         __syncthreads();
     }
     const int npos = pre ? kc + cnt[3] : kc;  // work items of this CTA
-    // work item at a position of the order: the head's item index and its half
-    auto item_at = [&](int pos, int &half) -> int {
-        half = 0;
+    // work item at a position of the order: the head's item index and its part
+    // (pinfo = part | parts << 4; 0 for a whole head)
+    auto item_at = [&](int pos, int &pinfo) -> int {
+        pinfo = 0;
         if (pos >= npos) return n_items;
         if (!pre) return bx + pos * G;
         const int o = order[pos];
-        half = o >> 10;
+        const int part = (o >> 10) & 7;
+        if (part) pinfo = part | ((1 << (o >> 13)) << 4);
         return bx + (o & 1023) * G;
     };
     // warps take the next position from a shared counter as they finish, so a warp
     // held up by a merge head takes fewer heads
-    auto grab = [&](int &half) -> int {
+    auto grab = [&](int &pinfo) -> int {
         int pos = 0;
         if (lane == 0) pos = atomicAdd(next_k, 1);
-        return item_at(__shfl_sync(FULL, pos, 0), half);
+        return item_at(__shfl_sync(FULL, pos, 0), pinfo);
     };
     const int E = p.E;
     const uint64_t pol_stream = ptx::policy_evict_first();
@@ -302,9 +328,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         if (pre) return pre_len[(hd.it - bx) / G];
         return p.log_len ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
     };
-    auto resolve_slot = [&](Head &hd, int it, int s, int half) {
+    auto resolve_slot = [&](Head &hd, int it, int s, int pinfo) {
         hd.it = it;
-        hd.half = half;
+        hd.part = pinfo & 15;
+        hd.np = pinfo >> 4;
         hd.s = s;
         hd.ok = 0;
         hd.c = 0;
@@ -332,7 +359,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         const bool merge = p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every));
         hd.mk = !merge ? MK_APPEND : c > TM_ENT ? MK_ROUNDS : DELTA ? MK_PASS2 : MK_FUSED;
         hd.nl = (c + EPC - 1) / EPC;
-        hd.n = hd.nl + (hd.half ? NCH / 2 : NCH) + (hd.mk == MK_PASS2 ? NCH : 0);
+        hd.n = hd.nl + (hd.part ? NCH / hd.np : NCH) + (hd.mk == MK_PASS2 ? NCH : 0);
     };
     // L2 warm-up of a head's token rows (they depend on the work item only)
     auto warm_token = [&](int it) {
@@ -354,11 +381,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     Head cur, nxt;
     nxt.ok = 0;
     nxt.n = 0;
-    int half0 = 0, half_nxt = 0;
-    const int it0 = item_at(w, half0);
+    int pinfo0 = 0, pinfo_nxt = 0;  // part info of the current and the next item
+    const int it0 = item_at(w, pinfo0);
     warm_token(it0);
-    resolve_slot(cur, it0, slot_of(it0), half0);
-    int it_nxt = grab(half_nxt);         // the warp's next head, and its slot id, one head early
+    resolve_slot(cur, it0, slot_of(it0), pinfo0);
+    int it_nxt = grab(pinfo_nxt);         // the warp's next head, and its slot id, one head early
     int s_nxt = slot_of(it_nxt);
     bool nxt_res = false;                // nxt's live length known
     int c_nxt = 0;
@@ -379,7 +406,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     ptx::bulk_g2s(dst + (size_t)(i - lo) * ESF, src + (size_t)i * E, ESB, bar, pol_stream);
             }
         } else {
-            const int y = x - hd.nl + (hd.half == 2 ? NCH / 2 : 0);   // the upper half starts at row 64
+            const int y = x - hd.nl + (hd.part ? (hd.part - 1) * (NCH / hd.np) : 0);  // a part's first chunk
             const bool keep = y < NCH && (hd.mk == MK_PASS2 || hd.mk == MK_ROUNDS);
             ptx::mbar_arrive_expect_tx(bar, CB);
             ptx::bulk_g2s(dst, p.state + hd.head * (size_t)(DK * DV) + (size_t)(y & (NCH - 1)) * CF, CB, bar,
@@ -407,7 +434,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     };
     // wait for stream position gc; false when the wait ran out (warp-uniform)
     auto wait_chunk = [&]() -> bool {
-        const bool ok = ptx::mbar_wait_bounded(&fb[gc % NSW], (gc / NSW) & 1, p.wait_ns);
+        const bool ok = ptx::mbar_wait_bounded(&fb[gc % NSW], (gc / NSW) & 1, WAIT_NS);
         return __all_sync(FULL, ok);
     };
     // done reading stream position gc: free its stage and keep the ring full
@@ -436,9 +463,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     };
 
     while (cur.it < n_items) {
+        if (p.stall_ns && bx == 0 && w == 0 && gc == 0) {
+            // timeout test: a wait that runs out, with the warp's first copies in flight
+            const bool ok = ptx::mbar_wait_bounded(stall_bar, 0u, p.stall_ns);
+            if (!__all_sync(FULL, ok)) { abort = true; break; }
+        }
         // the next head: slot id read one head ago; its live length is loaded now
         // and used when the stream reaches it
-        resolve_slot(nxt, it_nxt, s_nxt, half_nxt);
+        resolve_slot(nxt, it_nxt, s_nxt, pinfo_nxt);
         nxt_res = false;
         c_nxt = len_of(nxt);
         if (nxt.ok) warm_token(nxt.it);
@@ -569,7 +601,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
             if (abort) break;
             if (stage_tm) ptx::tmem_wait_st();
-            if (cur.half == 2) Yq = make_float4(0.f, 0.f, 0.f, 0.f);  // counted once, by the lower half
+            if (cur.part > 1) Yq = make_float4(0.f, 0.f, 0.f, 0.f);  // counted once, by the first part
 
             // new rows of one 16-row block of the merged state from its Sbar rows in
             // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending.
@@ -630,7 +662,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             // -- AppendDecode pass 1: y_q = Sbar^T qt, y_k = Sbar^T kt (columns 4l..4l+3);
             //    without the delta rule a merge writes its new rows here as well
             const float4 v4 = make_float4(v_own[0], v_own[1], v_own[2], v_own[3]);
-            const int cx0 = cur.half == 2 ? NCH / 2 : 0, cx1 = cur.half == 1 ? NCH / 2 : NCH;
+            const int cx0 = cur.part ? (cur.part - 1) * (NCH / cur.np) : 0;
+            const int cx1 = cur.part ? cx0 + NCH / cur.np : NCH;
             for (int cx = cx0; cx < cx1; ++cx) {
                 if (!wait_chunk()) { abort = true; break; }
                 const float *sb = st + (size_t)(gc % NSW) * CF;
@@ -667,35 +700,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
             const float4 bt4 = make_float4(bt[0], bt[1], bt[2], bt[3]);
             bool commits = true;  // this work item finalizes the head
-            if (cur.half) {
-                // Split merge: the first half to finish leaves its partial (its rows'
-                // share of Sbar^T qt; the lower half also the replay) in out and marks
-                // it; the second adds it to its own and the token term, and commits.
-                float4 *orow = reinterpret_cast<float4 *>(p.out + row * DV) + lane;
+            if (cur.part) {
+                // Split merge: every part adds its partial (its rows' share of
+                // Sbar^T qt; the first part also the replay) into the head's
+                // shared-memory accumulator and counts itself in; the last to arrive
+                // adds the token term, writes o_t and commits the head.
                 int *cm = comb + (cur.it - bx) / G;
-                int first = 0;
-                if (lane == 0) first = atomicAdd(cm, 1);
-                first = __shfl_sync(FULL, first, 0);
-                if (first == 0) {
-                    *orow = Yq;
-                    __threadfence();
-                    __syncwarp();
-                    if (lane == 0) atomicAdd(cm, 4);  // partial ready (arrivals count 1, 2)
-                    commits = false;
+                // the accumulator index (high bits) is fixed since the head list was built
+                float *acc = pacc + (size_t)((*reinterpret_cast<volatile int *>(cm) >> 8) - 1) * DV + 4 * lane;
+                atomicAdd(acc + 0, Yq.x);
+                atomicAdd(acc + 1, Yq.y);
+                atomicAdd(acc + 2, Yq.z);
+                atomicAdd(acc + 3, Yq.w);
+                __threadfence_block();
+                __syncwarp();
+                int prior = 0;
+                if (lane == 0) prior = atomicAdd(cm, 1) & 0xff;
+                prior = __shfl_sync(FULL, prior, 0);
+                if (prior == cur.np - 1) {
+                    __threadfence_block();
+                    const float4 tot = *reinterpret_cast<const float4 *>(acc);
+                    *reinterpret_cast<float4 *>(p.out + row * DV + 4 * lane) =
+                        make_float4(fmaf(bt[0], kq, tot.x), fmaf(bt[1], kq, tot.y),
+                                    fmaf(bt[2], kq, tot.z), fmaf(bt[3], kq, tot.w));
                 } else {
-                    // the other half is past its atomic and stores its partial next
-                    bool ready = false;
-                    if (lane == 0) {
-                        const uint64_t t0 = ptx::globaltimer_ns();
-                        while (!(ready = (atomicAdd(cm, 0) & 4) != 0)) {
-                            if (ptx::globaltimer_ns() - t0 > p.wait_ns) break;
-                        }
-                    }
-                    ready = __shfl_sync(FULL, ready ? 1 : 0, 0) != 0;
-                    if (!ready) { abort = true; break; }
-                    __threadfence();
-                    const float4 other = __ldcg(orow);
-                    *orow = make_float4(o[0] + other.x, o[1] + other.y, o[2] + other.z, o[3] + other.w);
+                    commits = false;
                 }
             } else if (p.want_out) {
                 *reinterpret_cast<float4 *>(p.out + row * DV + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
@@ -781,7 +810,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     __syncwarp();
                     for (int cx = 0; cx < NCH; ++cx) {
                         const uint32_t bb = cx & 1;
-                        const bool ok = ptx::mbar_wait_bounded(&pb[bb], (pph >> bb) & 1u, p.wait_ns);
+                        const bool ok = ptx::mbar_wait_bounded(&pb[bb], (pph >> bb) & 1u, WAIT_NS);
                         if (!__all_sync(FULL, ok)) { abort = true; break; }
                         pph ^= 1u << bb;
                         pb_pend &= ~(1u << bb);
@@ -824,7 +853,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
             // -- Finalize: the last unit of the (slot, layer) commits the live length
             //    (the atomic is issued now, its result looked at one head later)
-            if (!p.eager && commits) {
+            // (a merge from an empty log leaves it empty: nothing to commit, and every
+            //  unit of the slot saw the same c, so none of them counts itself in)
+            if (!p.eager && commits && !(mk != MK_APPEND && c == 0)) {
                 if (lane == 0) fin_old = atomicAdd(p.arrive + sl, 1);
                 fin_sl = sl;
                 fin_len = mk != MK_APPEND ? 0 : c + 1;
@@ -840,7 +871,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         cur = nxt;
         nxt.ok = 0;
         nxt.n = 0;
-        it_nxt = grab(half_nxt);
+        it_nxt = grab(pinfo_nxt);
         s_nxt = slot_of(it_nxt);
         nxt_res = false;
         issue_upto(gc + NSW);

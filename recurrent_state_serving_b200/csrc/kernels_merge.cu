@@ -69,6 +69,36 @@ cudaError_t launch_clear_bits(int32_t *err, int32_t bits, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+namespace {
+
+template <int DECAY>
+cudaError_t merge_head_one(const KParams &p, bool materialize, cudaStream_t st) {
+    const size_t smem = (size_t)2 * p.L * 128 * sizeof(float);
+    auto kern = merge_head_kernel<DECAY>;
+    static bool configured = false;  // per instantiation: room for the largest log (64 entries)
+    if (!configured) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   2 * 64 * 128 * (int)sizeof(float));
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const long long grid = (long long)p.batch * p.H;
+    kern<<<(unsigned)grid, MH_NT, smem, st>>>(p, materialize ? 1 : 0);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_merge_head(const KParams &p, int decay, bool materialize, cudaStream_t st) {
+    if (p.dk != 128 || p.dv != 128) return cudaErrorInvalidValue;
+    switch (decay) {
+    case DL_DECAY_NONE: return merge_head_one<DL_DECAY_NONE>(p, materialize, st);
+    case DL_DECAY_SCALAR: return merge_head_one<DL_DECAY_SCALAR>(p, materialize, st);
+    case DL_DECAY_DIAG: return merge_head_one<DL_DECAY_DIAG>(p, materialize, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_merge(const KParams &p, int bv, int decay, bool materialize, cudaStream_t st) {
     if (p.dk == 16 && bv == 16) return merge_decay<16, 16>(p, decay, materialize, st);
     if (p.dk == 64 && bv == 16) return merge_decay<64, 16>(p, decay, materialize, st);

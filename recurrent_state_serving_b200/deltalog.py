@@ -77,13 +77,13 @@ _lib.dl_reset_slots.argtypes = [_vp, _vp, ctypes.c_int32, _vp]
 _lib.dl_read_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, _vp]
 _lib.dl_decode_step_noalloc.argtypes = [ctypes.POINTER(dl_pool_desc), ctypes.c_int32,
                                         ctypes.POINTER(dl_step_args), ctypes.c_int32, _vp]
-_lib.dl_debug_wait_limit.argtypes = [ctypes.c_int64]
+_lib.dl_debug_stall.argtypes = [ctypes.c_int64]
 _lib.dl_merge_policy.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
 _lib.dl_status_string.argtypes = [ctypes.c_int]
 _lib.dl_status_string.restype = ctypes.c_char_p
 for _f in ("dl_log_bytes", "dl_create_pool", "dl_destroy_pool", "dl_decode_step", "dl_append", "dl_eager_step",
            "dl_merge", "dl_materialize", "dl_reset_slots", "dl_read_error", "dl_decode_step_noalloc",
-           "dl_debug_wait_limit", "dl_merge_policy"):
+           "dl_debug_stall", "dl_merge_policy"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -303,10 +303,11 @@ def dl_merge_policy(batch: int, n_heads: int, auto_merge="adaptive") -> bool:
     return bool(out.value)
 
 
-def dl_debug_wait_limit(limit_ns: int = 0):
-    """Test hook: bound of the whole-head kernel's pipeline waits for later launches
-    (process-wide); limit_ns <= 0 restores the default 100 ms."""
-    _check(_lib.dl_debug_wait_limit(int(limit_ns)), "dl_debug_wait_limit")
+def dl_debug_stall(limit_ns: int = 0):
+    """Test hook: while limit_ns > 0, each whole-head decode launch makes one warp wait
+    (bounded by limit_ns) on a barrier nothing completes, so it takes the kernel's
+    timeout path; limit_ns <= 0 switches it off (process-wide)."""
+    _check(_lib.dl_debug_stall(int(limit_ns)), "dl_debug_stall")
 
 
 class PreparedStep:

@@ -60,22 +60,27 @@ def stack_inputs(wl: synth.Workload, seq: list, rows) -> dict:
 
 
 def oracle_reference(wl: synth.Workload, layer: int, T: int, rows=None, ckpts=(), update=None,
-                     main_inputs=None):
+                     main_inputs=None, main_selected=False):
     """Eager fp64 reference for the rows' main steps 0..T-1 (after their staggering
-    pre-steps).  ckpts count main steps (0 = after the pre-steps).
+    pre-steps).  ckpts count main steps (0 = after the pre-steps).  main_inputs: the
+    main steps' step_inputs() dicts (full batch, or only `rows` when main_selected).
     Returns O [T, R, H, d_v], S [len(ckpts), R, H, d_k, d_v]."""
     rows = np.arange(wl.batch) if rows is None else np.asarray(rows)
     update = update or wl.update
     offs = synth.slot_offsets(wl)[rows]
     S0 = synth.initial_state(wl, layer)[rows].astype(np.float64)
-    main = main_inputs if main_inputs is not None else [synth.step_inputs(wl, t, layer) for t in range(T)]
-    pre = [synth.step_inputs(wl, p, layer, prestep=True) for p in range(int(offs.max()))]
+    sel = lambda x: synth.select_rows(wl, x, rows)
+    if main_inputs is None:
+        main = [sel(synth.step_inputs(wl, t, layer)) for t in range(T)]
+    else:
+        main = list(main_inputs) if main_selected else [sel(x) for x in main_inputs]
+    pre = [sel(synth.step_inputs(wl, p, layer, prestep=True)) for p in range(int(offs.max()))]
     R = len(rows)
     O = np.zeros((T, R, wl.n_heads, wl.d_v))
     S = np.zeros((len(ckpts), R, wl.n_heads, wl.d_k, wl.d_v))
     for o in np.unique(offs):
         idx = np.nonzero(offs == o)[0]
-        x = stack_inputs(wl, pre[:o] + main, rows[idx])
+        x = stack_inputs(wl, pre[:o] + main, idx)
         Oo, So = oracle.eager_rollout(S0[idx], x["Q"], x["K"], x["V"], x["LAM"], x["BETA"],
                                       decay=wl.decay, update=update,
                                       lambda_const=wl.lambda_const,
@@ -85,10 +90,14 @@ def oracle_reference(wl: synth.Workload, layer: int, T: int, rows=None, ckpts=()
     return O, S
 
 
-def gpu_rollout(runner: DecodeRunner, T: int, ckpts=(), layers=None, keep_inputs=False):
+def gpu_rollout(runner: DecodeRunner, T: int, ckpts=(), layers=None, keep_inputs=False, state_rows=None,
+                out_rows=None):
     """Run T common steps (after set-up and pre-steps) on the GPU.
     Returns ({layer: O [T, B, H, d_v]}, {layer: S [len(ckpts), B, H, d_k, d_v]},
-    {layer: [host inputs per step]})."""
+    {layer: [host inputs per step]}).  state_rows / out_rows: keep only these batch
+    rows of the checkpointed states / outputs (the device still runs every row); with
+    out_rows the kept inputs hold only those rows too (oracle_reference(...,
+    main_selected=True))."""
     layers = runner.layers if layers is None else layers
     wl = runner.wl
     runner.load_initial_state()
@@ -96,18 +105,28 @@ def gpu_rollout(runner: DecodeRunner, T: int, ckpts=(), layers=None, keep_inputs
     outs = {l: [] for l in layers}
     states = {l: [] for l in layers}
     kept = {l: [] for l in layers}
+    sel = None if state_rows is None else torch.as_tensor(np.asarray(state_rows), device=runner.device)
+    osel = None if out_rows is None else torch.as_tensor(np.asarray(out_rows), device=runner.device)
+
+    def snap(l):
+        S = runner.materialize(l)
+        if sel is not None:
+            S = S.index_select(0, sel)
+        return S.double().cpu().numpy()
     for l in layers:
         if 0 in ckpts:
-            states[l].append(runner.materialize(l).double().cpu().numpy())
+            states[l].append(snap(l))
     for t in range(T):
         for l in layers:
             host = synth.step_inputs(wl, t, l)
             if keep_inputs:
-                kept[l].append(host)
+                kept[l].append(host if out_rows is None else synth.select_rows(wl, host, np.asarray(out_rows)))
             o = runner.call(l, runner.device_inputs(host))
+            if osel is not None:
+                o = o.index_select(0, osel)
             outs[l].append(o.double().cpu().numpy())
             if t + 1 in ckpts:
-                states[l].append(runner.materialize(l).double().cpu().numpy())
+                states[l].append(snap(l))
     torch.cuda.synchronize()
     return ({l: np.stack(v) for l, v in outs.items()},
             {l: (np.stack(v) if v else None) for l, v in states.items()}, kept)

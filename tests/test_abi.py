@@ -9,7 +9,7 @@ import torch
 
 from recurrent_state_serving_b200 import deltalog as dl
 
-EXPECTED = ["dl_append", "dl_create_pool", "dl_debug_wait_limit", "dl_decode_step", "dl_decode_step_noalloc",
+EXPECTED = ["dl_append", "dl_create_pool", "dl_debug_stall", "dl_decode_step", "dl_decode_step_noalloc",
             "dl_destroy_pool", "dl_eager_step", "dl_log_bytes", "dl_materialize", "dl_merge", "dl_merge_policy",
             "dl_read_error", "dl_reset_slots", "dl_status_string"]
 

@@ -204,6 +204,7 @@ def test_sub_record_steps_and_specs():
     wl = bench.parse_spec("gla_rwkv6_diag:b64:L8")
     assert (wl.batch, wl.log_cap) == (64, 8)
     assert bench.parse_spec("retnet_scalar:b1024").batch == 1024
+    assert bench.parse_spec("kda_diag_delta:n1:b32").n_layers == 1
     with pytest.raises(SystemExit):
         bench.parse_spec("nope")
     with pytest.raises(SystemExit):

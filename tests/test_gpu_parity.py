@@ -149,17 +149,32 @@ def test_log_contents_match_the_deferred_oracle(tile_v, log_format):
                 np.testing.assert_allclose(ent[dk + dv:], ref.Lam_log[i], rtol=1e-5, atol=1e-7)
 
 
-def test_append_then_merge_flow():
-    """dl_append fills all L rows, dl_merge folds them, decode continues."""
-    wl = synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=30, log_cap=5)
-    r = DecodeRunner(wl, n_slots=6, slot_seed=3)
+MERGE_FLOW = {
+    "kda": synth.KDA.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=30, log_cap=5),
+    "retnet": synth.RETNET.with_(n_layers=1, batch=3, n_heads=4, n_kheads=4, steps=30, log_cap=5,
+                                 staggered=False),
+    "la_d128": REDUCED["la_d128"].with_(steps=30, log_cap=5),
+    "gla_L64": synth.GLA_DIAG.with_(batch=2, n_heads=3, n_kheads=3, steps=140, log_cap=64),
+}
+
+
+@pytest.mark.parametrize("log_format", ["fp32", "compact"])
+@pytest.mark.parametrize("tile_v", [0, 16])
+@pytest.mark.parametrize("name", sorted(MERGE_FLOW))
+def test_append_then_merge_flow(name, tile_v, log_format):
+    """dl_append fills all L rows, dl_merge folds them, decode continues; every state is
+    read back with dl_materialize (whole-head merge kernel for tile_v 0, value-tiled
+    for 16)."""
+    wl = MERGE_FLOW[name]
+    r = DecodeRunner(wl, n_slots=6, slot_seed=3, tile_v=tile_v, log_format=log_format)
     r.load_initial_state()
     T = wl.steps
     gpu_states = []
     for t in range(T):
         x = r.gen_inputs(t, 0)
         if t < 2 * wl.log_cap:   # append-only phase with explicit merges
-            dl.dl_append(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"])
+            dl.dl_append(r.pool, 0, r.slots, x["q"], x["k"], x["v"], lam=x["lam"], beta=x["beta"],
+                         lambda_per_head=wl.lambda_const)
             if (t + 1) % wl.log_cap == 0:
                 assert int(r.pool.log_len[r.slots.long(), 0].min()) == wl.log_cap
                 dl.dl_merge(r.pool, 0, r.slots)
@@ -286,15 +301,58 @@ def test_fullsize_gla_all_heads(log_cap):
 
 
 def test_fullsize_kda_sampled_rows():
+    """KDA at full size (24 layers x 256 slots x 32 heads, L = 16, 64 steps): sampled
+    rows of the first and last layer, outputs at every step and the logical state
+    (dl_materialize) after step 32 and step 64."""
     wl = synth.KDA
     rows = np.array([0, 77, 160, 255])
     layers = [0, wl.n_layers - 1]
+    ck = [wl.steps // 2, wl.steps]
     r = DecodeRunner(wl, layers=layers)
-    outs, _, kept = H.gpu_rollout(r, wl.steps, keep_inputs=True)
+    outs, states, kept = H.gpu_rollout(r, wl.steps, ckpts=ck, keep_inputs=True, state_rows=rows,
+                                       out_rows=rows)
     assert r.errors() == 0
     for l in layers:
-        O, _ = H.oracle_reference(wl, l, wl.steps, rows=rows, main_inputs=kept[l])
-        H.check_steps(outs[l][:, rows], O)
+        O, S = H.oracle_reference(wl, l, wl.steps, rows=rows, ckpts=ck, main_inputs=kept[l], main_selected=True)
+        H.check_steps(outs[l], O)
+        H.check_steps(states[l], S, elem=None, what=f"KDA layer {l} state")
+    del r
+    torch.cuda.empty_cache()
+
+
+def test_fullsize_retnet_b256_every_layer_staggered():
+    """RetNet as benchmarked: 8 layers x 256 slots x 32 heads, L = 32, staggered merge
+    phases, 128 steps; sampled rows on every layer, outputs at every step and the
+    logical state after the last step."""
+    wl = synth.RETNET
+    rows = np.array([3, 128, 250])
+    T = wl.steps
+    r = DecodeRunner(wl)
+    outs, states, kept = H.gpu_rollout(r, T, ckpts=[T], keep_inputs=True, state_rows=rows, out_rows=rows)
+    assert r.errors() == 0
+    for l in r.layers:
+        O, S = H.oracle_reference(wl, l, T, rows=rows, ckpts=[T], main_inputs=kept[l], main_selected=True)
+        H.check_steps(outs[l], O, what=f"RetNet layer {l} output")
+        H.check_steps(states[l], S, elem=None, what=f"RetNet layer {l} state")
+    del r
+    torch.cuda.empty_cache()
+
+
+def test_more_heads_than_the_head_list_holds():
+    """131,072 heads in one launch: each CTA has more heads than its head list holds
+    (512 per CTA at 148 SMs), so heads are neither ordered nor split.  Staggered
+    merges happen inside the window; sampled rows against the oracle."""
+    wl = synth.RETNET.with_(n_layers=1, batch=4096, steps=12)
+    rows = np.array([0, 2047, 4095])
+    T = wl.steps
+    r = DecodeRunner(wl, tile_v=128)
+    outs, states, kept = H.gpu_rollout(r, T, ckpts=[T], keep_inputs=True, state_rows=rows, out_rows=rows)
+    assert r.errors() == 0
+    offs = synth.slot_offsets(wl)
+    assert ((offs + T) >= wl.log_cap).any()   # some slots merge inside the window
+    O, S = H.oracle_reference(wl, 0, T, rows=rows, ckpts=[T], main_inputs=kept[0], main_selected=True)
+    H.check_steps(outs[0], O)
+    H.check_steps(states[0], S, elem=None, what="state")
     del r
     torch.cuda.empty_cache()
 
@@ -403,14 +461,25 @@ def test_cluster_replay_matches_per_tile_bit_for_bit(name, tile_v):
         np.testing.assert_array_equal(res["cluster"][1][layer], res["per_tile"][1][layer])
 
 
-# ---- merge heads split in two halves (CTAs with more heads than warps) ---------------
+# ---- merge heads split into 2 or 4 parts (CTAs with fewer than 24 heads) ---------------
+# (batch, heads, L): 3200 heads (21-22 per CTA, halves at c < 16); 2048 heads with
+# L = 32 (13-14 per CTA, quarters); 1024 heads (6-7 per CTA, halves over the idle
+# warps); 592 heads (4 per CTA, quarters); L = 17 (c = 16: quarters at 21-22 per CTA).
+SPLIT_SHAPES = {"b200_h16_L4": (200, 16, 4), "b64_h32_L32": (64, 32, 32), "b64_h16_L8": (64, 16, 8),
+                "b37_h16_L8": (37, 16, 8), "b200_h16_L17": (200, 16, 17)}
+
+
+@pytest.mark.parametrize("shape", sorted(SPLIT_SHAPES))
 @pytest.mark.parametrize("staggered,log_format", [(False, "fp32"), (True, "fp32"), (True, "compact")])
-def test_split_merge_heads_match_the_oracle(staggered, log_format):
-    """3200 heads over at most 148 CTAs: every CTA orders its heads and splits each merge
-    without the delta rule into two half-tile work items whose partial outputs combine.
-    Non-staggered, every slot merges at once (all heads split); staggered, a few do."""
-    wl = synth.GLA_DIAG.with_(batch=200, steps=24, log_cap=4, staggered=staggered)
-    rows = np.array([0, 77, 199])
+def test_split_merge_heads_match_the_oracle(shape, staggered, log_format):
+    """Every CTA with fewer than 24 heads orders its heads and splits each merge without
+    the delta rule into 2 or 4 row-range work items whose partial outputs combine in
+    shared memory.  Non-staggered, every slot merges at once (every merge head is split,
+    as far as the CTA's accumulators go); staggered, a few do."""
+    B, Hh, L = SPLIT_SHAPES[shape]
+    wl = synth.GLA_DIAG.with_(batch=B, n_heads=Hh, n_kheads=Hh, steps=L * 2 + 5, log_cap=L,
+                              staggered=staggered)
+    rows = np.array([0, B // 2 - 1, B - 1])
     r = DecodeRunner(wl, tile_v=128, log_format=log_format)
     T = wl.steps
     outs, states, kept = H.gpu_rollout(r, T, ckpts=[T], keep_inputs=True)
@@ -426,20 +495,21 @@ def test_split_merge_heads_match_the_oracle(staggered, log_format):
 
 
 def test_expired_wait_sets_the_timeout_bit_and_the_pool_recovers():
-    """A pipeline wait of the whole-head kernel made to run out (test hook: a 1 ns
-    limit) sets DL_EBIT_TIMEOUT; the kernel drains its own copies and returns, the
+    """A wait of the whole-head kernel made to run out (test hook: one warp waits, for
+    at most 2 ms, on a barrier nothing completes, with its first bulk copies in
+    flight) sets DL_EBIT_TIMEOUT; the kernel drains its own copies and returns, the
     context stays usable, and after a fresh prefill and reset the same pool matches
     the oracle again."""
     wl = synth.GLA_DIAG.with_(batch=16, n_heads=16, n_kheads=16, steps=12, log_cap=4)
     r = DecodeRunner(wl, tile_v=128)
     r.load_initial_state()
-    dl.dl_debug_wait_limit(1)
+    dl.dl_debug_stall(2_000_000)
     try:
         for t in range(2 * wl.log_cap):   # append steps and merge steps
             r.call(0, r.gen_inputs(t, 0))
         bits = dl.dl_read_error(r.pool, clear=False)
     finally:
-        dl.dl_debug_wait_limit(0)
+        dl.dl_debug_stall(0)
     assert bits & dl.DL_EBIT_TIMEOUT, f"error bits {bits:#x}"
     assert dl.dl_read_error(r.pool, clear=True) == bits      # read, then cleared
     assert dl.dl_read_error(r.pool) == 0
