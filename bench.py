@@ -67,7 +67,8 @@ ROTATE_MIN_BYTES = 384 << 20  # base-state bytes of one rotation: three times L2
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 CSRC = os.path.join(ROOT, "recurrent_state_serving_b200", "csrc")
 DEFAULT_WORKLOAD = "kda_diag_delta"
-DEFAULT_SUBS = "gla_rwkv6_diag:b64:L8,retnet_scalar:b64,retnet_scalar:b256,retnet_scalar:b1024,gdn_gva:b1"
+DEFAULT_SUBS = ("gla_rwkv6_diag:b64:L8,retnet_scalar:b64,retnet_scalar:b256,retnet_scalar:b1024,gdn_gva:b1,"
+                "retnet_scalar:b1,retnet_scalar:b16")
 DEFAULT_MERGE_LEGS = "kda_diag_delta,retnet_scalar:b256"
 SUB_MIN_MS = 3.0            # a sub-record's timed region is at least about this long
 SUB_MAX_STEPS = 4096
@@ -203,6 +204,16 @@ def group_live_entries(group_offsets, step_index: int, log_cap: int):
     """live_entries() with each group's own offsets ([n_groups, batch])."""
     R = group_offsets.shape[0]
     return (group_offsets[step_index % R] + step_index // R) % log_cap
+
+
+def expected_live_lengths(wl, group_offsets, n_steps: int, merge_every: bool = False):
+    """Live entries of every slot of every group ([n_groups, batch]) after global steps
+    0 .. n_steps-1 (step j on group j mod R), as the byte accounting assumes."""
+    R = group_offsets.shape[0]
+    taken = np.array([(n_steps - g + R - 1) // R for g in range(R)])
+    if merge_every:
+        return np.zeros_like(group_offsets)
+    return (group_offsets + taken[:, None]) % wl.log_cap
 
 
 def timed_window_bytes(wl, group_offsets, first: int, K: int, log_format: str = "fp32",
@@ -675,6 +686,11 @@ def decode_leg(ctx, wl, K, W, setup, merge):
     total_ms = ctx.timed(prepared_calls("decode", wl, r, setup, R, {}, merge), K, W)
     if r.errors() != 0:
         raise RuntimeError("device error bits set during the benchmark")
+    # the slots' live lengths must be the ones the byte accounting assumes
+    live = np.stack([r.pool.log_len[gs.long(), 0].cpu().numpy() for gs in r.group_slots])
+    want = expected_live_lengths(wl, goffs, W + K, every)
+    if not np.array_equal(live, want):
+        raise RuntimeError(f"slot phases differ from the byte model in {int((live != want).sum())} slots")
     max_ms = ctx.reduce_max(total_ms)
     launches = K * wl.n_layers
     ctx.launches += launches

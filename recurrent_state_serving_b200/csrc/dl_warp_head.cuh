@@ -37,11 +37,17 @@
 // (pass-1 copies ask L2 to keep it).  Logs longer than TM_ENT entries (log_cap > 32)
 // merge in rounds of MRB entries staged in shared memory instead.
 //
-// Order of work.  The CTA's heads are blockIdx.x + k * gridDim.x.  When there are more
-// of them than warps (and at most KMAX), the CTA first reads every head's slot id and
-// live length (all threads at once) and puts the merge steps first: a merge head
-// costs several append heads, and started early it overlaps their streaming instead
-// of ending the launch alone.  When the CTA has few heads, a merge without the delta
+// Order of work.  Which heads a CTA takes: with a batch of at most BAL_ROWS slots on a
+// decode step that can merge, and one to three heads per warp (where a CTA's merges
+// decide its time), every CTA reads the whole batch's slot ids and live
+// lengths (all threads at once, one load each) and applies the same rule: the merge
+// heads of the launch are dealt round-robin over the CTAs, and each CTA takes a
+// contiguous share of the append heads sized so that every CTA's cost (a merge head
+// counted as 2 + (L-1)/16 append heads) is about equal.  Otherwise the CTA's heads are
+// blockIdx.x + k * gridDim.x.  With more than one head (and at most KMAX), the CTA
+// reads its heads' slot ids and live lengths first and puts the merge steps first: a
+// merge head costs several append heads, and started early it overlaps their
+// streaming instead of ending the launch alone.  When the CTA has few heads, a merge without the delta
 // rule is split into 2 or 4 work items, each streaming and rewriting its share of the
 // tile's rows (each stages the coefficients in its own TMEM share) and adding its
 // partial output into a shared-memory accumulator of the head; the last part to
@@ -86,13 +92,18 @@ constexpr int AG = 4;                       // merge entries per TMEM load / sha
 // per-warp scratch: the head's row vectors qt, kt, e^{lbar_t}, k, lbar_t (5 x 128 floats)
 // and the A' values of AG entries for the 16 rows of one block
 constexpr int WSCR = 5 * DK + AG * CR;
-// per-CTA head list: slot id, live length, split combine state of up to KMAX heads,
-// and the processing order (a head split in S parts takes S positions)
-constexpr int KMAX = 512;
+// per-CTA head list: item index, slot id, live length, split combine state of up to
+// KMAX heads, and the processing order (a head split in S parts takes S positions)
+constexpr int KMAX = 256;
 constexpr int MAX_PARTS = 4;                // parts of a split merge head
 constexpr int NPA = 8;                      // split heads in flight per CTA (accumulators)
+// balanced schedule: the whole batch's slot ids and live lengths, and a bitmap of its
+// merging rows with per-word prefix counts
+constexpr int BAL_ROWS = 512;
+constexpr int BAL_WORDS = BAL_ROWS / 32;
 constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4 + (size_t)NW * NB * 8 + 32 +
-                        (size_t)KMAX * (4 + 4 + 4) + (size_t)2 * KMAX * 2 + (size_t)NPA * DV * 4;
+                        (size_t)KMAX * (4 + 4 + 4 + 4) + (size_t)2 * KMAX * 2 + (size_t)NPA * DV * 4 +
+                        (size_t)BAL_ROWS * (4 + 1) + (size_t)BAL_WORDS * (4 + 4);
 static_assert(KMAX + (MAX_PARTS - 1) * NPA <= 2 * KMAX, "the order holds every head and every extra part");
 static_assert(SMEM <= 232448, "a CTA may use at most 227 KB of shared memory");
 static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
@@ -156,6 +167,7 @@ struct Head {
     int n;         // stream positions: nl + NCH (+ NCH for MK_PASS2); 0 when skipped
     int part;      // 0: the whole head; 1..np: rows (part-1)*128/np .. part*128/np - 1 of a split merge
     int np;        // parts of a split merge head
+    int k;         // place in the CTA's head list (when there is one)
     size_t head;   // (slot, layer, head) index
 };
 
@@ -205,12 +217,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     int *next_k = reinterpret_cast<int *>(bars + (size_t)NW * NB * 8);
     uint32_t *tm_slot = reinterpret_cast<uint32_t *>(next_k + 1);
     int *cnt = next_k + 2;  // merge positions, next merge position, next other position, extra parts,
-                            // accumulators taken
-    int *pre_slot = next_k + 8;
+                            // accumulators taken, merging rows of the batch (balanced schedule)
+    int *pre_it = next_k + 8;    // item index (batch row * H + head) of the CTA's k-th head
+    int *pre_slot = pre_it + KMAX;
     int *pre_len = pre_slot + KMAX;
     int *comb = pre_len + KMAX;  // split merge heads: (accumulator + 1) << 8 | parts arrived
     uint16_t *order = reinterpret_cast<uint16_t *>(comb + KMAX);  // k | part << 10 | log2(parts) << 13
     float *pacc = reinterpret_cast<float *>(order + 2 * KMAX);  // NPA x DV partial outputs
+    int *row_slot = reinterpret_cast<int *>(pacc + NPA * DV);   // balanced schedule: per batch row
+    unsigned *bmap = reinterpret_cast<unsigned *>(row_slot + BAL_ROWS);  // merging rows
+    int *wpre = reinterpret_cast<int *>(bmap + BAL_WORDS);      // set bits before each word
+    uint8_t *row_len = reinterpret_cast<uint8_t *>(wpre + BAL_WORDS);
 
     // merges with live entries need tensor memory (auto-merge decode steps only)
     const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
@@ -223,6 +240,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         cnt[0] = cnt[1] = cnt[2] = cnt[3] = cnt[4] = 0;
     }
     for (int i = threadIdx.x; i < NPA * DV; i += NTHREADS) pacc[i] = 0.f;
+    for (int i = threadIdx.x; i < BAL_WORDS; i += NTHREADS) bmap[i] = 0u;
     if (use_tm && w == 0) {
         ptx::tmem_alloc(tm_slot, TM_COLS);
         ptx::tmem_relinquish();
@@ -242,13 +260,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
     const int n_items = p.batch * p.H;
     const int G = gridDim.x, bx = blockIdx.x;
-    const int kc = bx < n_items ? (n_items - 1 - bx) / G + 1 : 0;  // heads of this CTA
-    // the head list is built when there is an order to choose (more heads than warps)
-    // or spare warps to split a merge head over
-    const bool pre = kc > 1 && kc <= KMAX;
     auto merges = [&](int s, int c) {
         return s >= 0 && s < p.n_slots && (p.eager || (p.auto_merge && (c >= p.L - 1 || p.merge_every)));
     };
+    int kc = bx < n_items ? (n_items - 1 - bx) / G + 1 : 0;  // heads of this CTA (natural order)
+    // Balanced schedule (see the header): a decode step that can merge, with at most
+    // BAL_ROWS rows and one to three heads per warp on average.  With fewer, a CTA's
+    // time is its slowest warp, and the natural assignment already gives each CTA at
+    // most one item per warp.  With more, the merges of a CTA are a small part of its
+    // work and the natural, strided assignment streams faster: at any moment the
+    // whole GPU reads a window of consecutive heads, where contiguous per-CTA ranges
+    // spread the reads over the whole state (measured on B200: KDA, 55 heads per CTA,
+    // 0.80 against 0.86 of the copy rate).
+    bool bal = !p.eager && p.auto_merge && p.log_len && p.batch <= BAL_ROWS &&
+               (long long)n_items >= (long long)G * NW && (long long)n_items < (long long)G * 3 * NW;
+    if (bal) {
+        // every batch row's slot id and live length; merging rows set their bit
+        constexpr int RPT = BAL_ROWS / NTHREADS;
+        int sv[RPT];
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int b = threadIdx.x + j * NTHREADS;
+            sv[j] = b < p.batch ? p.slots[b] : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int b = threadIdx.x + j * NTHREADS;
+            if (b >= p.batch) continue;
+            const bool ok = sv[j] >= 0 && sv[j] < p.n_slots;
+            const int c = ok ? p.log_len[(size_t)sv[j] * p.n_layers + p.layer] : 0;
+            row_slot[b] = sv[j];
+            row_len[b] = (uint8_t)(c < 0 ? 255 : c > 254 ? 254 : c);  // out of [0, L]: flagged at the head
+            if (ok && merges(sv[j], c)) atomicOr(&bmap[b >> 5], 1u << (b & 31));
+        }
+        __syncthreads();
+        const int nwords = (p.batch + 31) >> 5;
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int i = 0; i < nwords; ++i) {
+                wpre[i] = acc;
+                acc += __popc(bmap[i]);
+            }
+            cnt[5] = acc;  // merging rows of the batch
+        }
+        __syncthreads();
+        // Integer costs in 1/16 of an append head (n_items <= G * KMAX / 4, so every
+        // quantity below fits 32 bits except the product in A()).  Nothing here loops
+        // over CTAs: this runs at the start of every launch.
+        const int NMH = cnt[5] * p.H, NA = n_items - NMH;
+        const int Wm = 32 + (p.L - 1);  // a merge head costs 2 + (L-1)/16 append heads
+        const int q = NMH / G, r = NMH % G;
+        const int target = (16 * NA + Wm * NMH) / G;
+        const int cap_lo = target > Wm * (q + 1) ? target - Wm * (q + 1) : 0;  // CTAs with q+1 merges
+        const int cap_hi = target > Wm * q ? target - Wm * q : 0;              // CTAs with q merges
+        auto P = [&](int x) -> long long {
+            return (long long)(x < r ? x : r) * cap_lo + (long long)(x > r ? x - r : 0) * cap_hi;
+        };
+        const long long PG = P(G);
+        auto A = [&](int x) -> int { return PG > 0 ? (int)((long long)NA * P(x) / PG) : (int)((long long)NA * x / G); };
+        // the same decision in every CTA: fall back unless every CTA's share fits the list
+        // (a CTA takes at most q + 1 merge heads and NA * cap / PG + 1 append heads)
+        const int cap_max = cap_lo > cap_hi ? cap_lo : cap_hi;
+        const long long kbound = q + 1 + (PG > 0 ? (long long)NA * cap_max / PG : (long long)NA / G) + 1;
+        if (kbound > KMAX) {
+            bal = false;
+        } else {
+            const int km = q + (bx < r ? 1 : 0);
+            const int a0 = A(bx);
+            kc = km + (A(bx + 1) - a0);
+            // row of the j-th merging / non-merging batch row
+            auto select = [&](int j, bool set) -> int {
+                int wd = 0;
+                auto before = [&](int i) -> int { return set ? wpre[i] : 32 * i - wpre[i]; };
+                while (wd + 1 < nwords && before(wd + 1) <= j) ++wd;
+                unsigned m = set ? bmap[wd] : ~bmap[wd];
+                for (int rem = j - before(wd); rem > 0; --rem) m &= m - 1;
+                return 32 * wd + __ffs(m) - 1;
+            };
+            for (int k = threadIdx.x; k < kc; k += NTHREADS) {
+                const int u = k < km ? bx + k * G : a0 + (k - km);  // merge / append head u of the launch
+                const int row = select(u / p.H, k < km);
+                pre_it[k] = row * p.H + u % p.H;
+                pre_slot[k] = row_slot[row];
+                pre_len[k] = row_len[row] == 255 ? -1 : row_len[row];
+            }
+        }
+    }
+    // the head list is built when there is an order to choose (more heads than warps),
+    // and always for the balanced schedule; with at most one head per warp each warp
+    // reads its own head's metadata, which measured faster than building the list
+    // (GLA B = 64: 0.66 against 0.74 of the copy rate with merges synchronised)
+    const bool pre = bal || (kc > NW && kc <= KMAX);
     // Merges written during pass 1 (no delta rule, at most TM_ENT entries) are split
     // when the CTA has few heads: a merge head costs several append heads (its
     // write-back is a chain of c-term updates run by one warp), so with fewer than
@@ -263,11 +365,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         return c >= 16 ? 4 : 2;
     };
     if (pre) {
+        if (!bal) {
+            for (int k = threadIdx.x; k < kc; k += NTHREADS) {
+                const int it = bx + k * G;
+                const int s = p.slots[it / p.H];
+                pre_it[k] = it;
+                pre_slot[k] = s;
+                pre_len[k] = (s >= 0 && s < p.n_slots && p.log_len) ? p.log_len[(size_t)s * p.n_layers + p.layer]
+                                                                     : 0;
+            }
+        }
+        __syncthreads();
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
-            const int s = p.slots[(bx + k * G) / p.H];
-            const int c = (s >= 0 && s < p.n_slots && p.log_len) ? p.log_len[(size_t)s * p.n_layers + p.layer] : 0;
-            pre_slot[k] = s;
-            pre_len[k] = c;
+            const int s = pre_slot[k], c = pre_len[k];
             int np = parts_of(s, c);
             int cm = 0;
             if (np > 1) {  // a split head needs one of the NPA accumulators
@@ -281,30 +391,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         }
         __syncthreads();
         const int nm = cnt[0];
+        // With many heads per warp (8 or more; no splits then, one position per head)
+        // and merges written during pass 1, the merge heads are spread evenly over all
+        // but the last NW positions: started all at once, their write-back (ALU work)
+        // would leave the SM with few streaming warps at the start of the launch
+        // (RetNet B = 1024: 0.905 -> 0.949 of the copy rate).  Otherwise they go first:
+        // with fewer heads the launch's tail must not end on a merge, and delta-rule
+        // merges, which re-read their tile from L2 in pass 2, measured slower spread
+        // (KDA: 0.86 -> 0.73).
+        const int span = kc - NW;
+        const bool spread = !DELTA && kc >= 8 * NW && nm > 0 && span >= nm;
+        auto merge_pos = [&](int i) { return spread ? (int)((long long)i * span / nm) : i; };
         for (int k = threadIdx.x; k < kc; k += NTHREADS) {
             const int s = pre_slot[k], c = pre_len[k];
             if (comb[k] != 0) {
                 const int np = parts_of(s, c), lg = np == 4 ? 2 : 1;
                 const int pos = atomicAdd(&cnt[1], np);  // the parts next to each other
                 for (int j = 0; j < np; ++j) order[pos + j] = (uint16_t)(k | ((j + 1) << 10) | (lg << 13));
+            } else if (merges(s, c)) {
+                order[merge_pos(atomicAdd(&cnt[1], 1))] = (uint16_t)k;
             } else {
-                const int pos = merges(s, c) ? atomicAdd(&cnt[1], 1) : nm + atomicAdd(&cnt[2], 1);
+                const int a = atomicAdd(&cnt[2], 1);
+                int pos = a;  // the a-th position no merge head takes
+                if (spread) {
+                    for (int i = 0; i < nm && merge_pos(i) <= pos; ++i) ++pos;
+                } else {
+                    pos += nm;
+                }
                 order[pos] = (uint16_t)k;
             }
         }
         __syncthreads();
     }
     const int npos = pre ? kc + cnt[3] : kc;  // work items of this CTA
-    // work item at a position of the order: the head's item index and its part
-    // (pinfo = part | parts << 4; 0 for a whole head)
+    // work item at a position of the order: the head's item index, its part and its
+    // place k in the CTA's list (pinfo = part | parts << 4 | k << 8; part 0: whole head)
     auto item_at = [&](int pos, int &pinfo) -> int {
         pinfo = 0;
         if (pos >= npos) return n_items;
         if (!pre) return bx + pos * G;
         const int o = order[pos];
-        const int part = (o >> 10) & 7;
-        if (part) pinfo = part | ((1 << (o >> 13)) << 4);
-        return bx + (o & 1023) * G;
+        const int part = (o >> 10) & 7, k = o & 1023;
+        pinfo = k << 8;
+        if (part) pinfo |= part | ((1 << (o >> 13)) << 4);
+        return pre_it[k];
     };
     // warps take the next position from a shared counter as they finish, so a warp
     // held up by a merge head takes fewer heads
@@ -319,19 +449,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 
     // -- head metadata: slot id first (it locates the tile and the log), live
     //    length after (it sizes the log part of the stream and decides the merge)
-    auto slot_of = [&](int it) -> int {
+    auto slot_of = [&](int it, int pinfo) -> int {
         if (it >= n_items) return -1;
-        return pre ? pre_slot[(it - bx) / G] : p.slots[it / p.H];
+        return pre ? pre_slot[pinfo >> 8] : p.slots[it / p.H];
     };
     auto len_of = [&](const Head &hd) -> int {
         if (!hd.ok) return 0;
-        if (pre) return pre_len[(hd.it - bx) / G];
+        if (pre) return pre_len[hd.k];
         return p.log_len ? p.log_len[(size_t)hd.s * p.n_layers + p.layer] : 0;
     };
     auto resolve_slot = [&](Head &hd, int it, int s, int pinfo) {
         hd.it = it;
         hd.part = pinfo & 15;
-        hd.np = pinfo >> 4;
+        hd.np = (pinfo >> 4) & 15;
+        hd.k = pinfo >> 8;
         hd.s = s;
         hd.ok = 0;
         hd.c = 0;
@@ -384,9 +515,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     int pinfo0 = 0, pinfo_nxt = 0;  // part info of the current and the next item
     const int it0 = item_at(w, pinfo0);
     warm_token(it0);
-    resolve_slot(cur, it0, slot_of(it0), pinfo0);
+    resolve_slot(cur, it0, slot_of(it0, pinfo0), pinfo0);
     int it_nxt = grab(pinfo_nxt);         // the warp's next head, and its slot id, one head early
-    int s_nxt = slot_of(it_nxt);
+    int s_nxt = slot_of(it_nxt, pinfo_nxt);
     bool nxt_res = false;                // nxt's live length known
     int c_nxt = 0;
 
@@ -705,7 +836,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                 // Sbar^T qt; the first part also the replay) into the head's
                 // shared-memory accumulator and counts itself in; the last to arrive
                 // adds the token term, writes o_t and commits the head.
-                int *cm = comb + (cur.it - bx) / G;
+                int *cm = comb + cur.k;
                 // the accumulator index (high bits) is fixed since the head list was built
                 float *acc = pacc + (size_t)((*reinterpret_cast<volatile int *>(cm) >> 8) - 1) * DV + 4 * lane;
                 atomicAdd(acc + 0, Yq.x);
@@ -872,7 +1003,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
         nxt.ok = 0;
         nxt.n = 0;
         it_nxt = grab(pinfo_nxt);
-        s_nxt = slot_of(it_nxt);
+        s_nxt = slot_of(it_nxt, pinfo_nxt);
         nxt_res = false;
         issue_upto(gc + NSW);
     }

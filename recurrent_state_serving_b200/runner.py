@@ -109,8 +109,9 @@ class DecodeRunner:
         return self.device_inputs(synth.step_inputs(self.wl, step, layer, prestep=prestep))
 
     # -- steps -----------------------------------------------------------------
-    def call(self, layer: int, x: dict, slots=None, out=None, stream=None):
-        """One library call for one layer (decode step or eager step)."""
+    def call(self, layer: int, x: dict, slots=None, out=None, stream=None, merge=None):
+        """One library call for one layer (decode step or eager step); merge overrides
+        the runner's merge policy for this call."""
         slots = self.slots if slots is None else slots
         if self.mode == "eager":
             return dl.dl_eager_step(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"],
@@ -118,12 +119,15 @@ class DecodeRunner:
                                     stream=stream)
         return dl.dl_decode_step(self.pool, layer, slots, x["q"], x["k"], x["v"], lam=x["lam"],
                                  beta=x["beta"], out=out, lambda_per_head=self.wl.lambda_const,
-                                 auto_merge=self.merge, stream=stream)
+                                 auto_merge=self.merge if merge is None else merge, stream=stream)
 
     def run_presteps(self, inputs=None):
         """Staggering: slot b of group g takes group_offsets[g, b] untimed decode steps
         first.  inputs(p, layer) -> device inputs of the whole batch for pre-step p
-        (default: the workload's own seeded pre-step inputs)."""
+        (default: the workload's own seeded pre-step inputs).  The pre-steps run on
+        sub-batches with the at-capacity merge policy whatever the runner's policy is:
+        the adaptive one would merge a small sub-batch on every step and undo the
+        staggering."""
         go = self.group_offsets
         n = int(go.max()) if go.size else 0
         for p in range(n):
@@ -142,7 +146,7 @@ class DecodeRunner:
                             x_all = inputs(p, layer)
                         x = self.select_device_rows(x_all, rows)
                     sel = torch.from_numpy(rows).to(self.device)
-                    self.call(layer, x, slots=gs[sel])
+                    self.call(layer, x, slots=gs[sel], merge="capacity")
 
     def select_device_rows(self, x: dict, rows) -> dict:
         """Rows of a device input dict (a per-head constant lambda is kept whole)."""

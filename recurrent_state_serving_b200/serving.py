@@ -75,14 +75,22 @@ class DecodeServer:
     ``log_cap="auto"`` takes the merge interval with the fewest modelled HBM bytes per
     head-step for this operator's shape, decay, update rule and log layout
     (``tuning.auto_log_cap``), which is the right choice when the batch fills the GPU.
+
+    ``merge`` is the library's merge policy: "capacity" (each slot merges on its L-th
+    step) or "adaptive" (as "capacity", but a batch too small to fill the GPU merges
+    every slot on every step, which is faster there; dl_merge_policy tells which).
     """
 
     def __init__(self, *, n_slots, n_layers, n_heads, d_k, d_v, log_cap, decay="none",
                  update="add", n_kheads=None, in_dtype=torch.bfloat16, lambda_per_head=False,
-                 log_format="fp32", tile_v=0, max_batch=None, device="cuda", use_graphs=True):
+                 log_format="fp32", tile_v=0, max_batch=None, device="cuda", use_graphs=True,
+                 merge="capacity"):
         if log_cap == "auto":
             log_cap = tuning.auto_log_cap(d_k, d_v, decay, update, log_format)
         self.log_cap = int(log_cap)
+        if merge not in ("capacity", "adaptive"):
+            raise ValueError("merge must be 'capacity' or 'adaptive'")
+        self.merge = merge
         self.pool = dl.Pool(n_slots, n_layers, n_heads, d_k, d_v, self.log_cap, decay=decay,
                             update=update, n_kheads=n_kheads, device=device, log_format=log_format,
                             tile_v=tile_v)
@@ -166,7 +174,7 @@ class DecodeServer:
                 lam = self.lam_const[l] if self.lambda_per_head else (None if b["lam"] is None else b["lam"][:B])
                 steps.append(dl.PreparedStep("decode", self.pool, l, self.slots_buf[:B], b["q"][:B], b["k"][:B],
                                              b["v"][:B], lam, None if b["beta"] is None else b["beta"][:B],
-                                             b["out"][:B], self.lambda_per_head))
+                                             b["out"][:B], self.lambda_per_head, auto_merge=self.merge))
             self._prepared[B] = steps
         return self._prepared[B]
 

@@ -237,3 +237,15 @@ def test_traffic_records_by_kind(tmp_path, monkeypatch):
     assert bench.recorded_traffic("w", "eager") == 20.0
     assert bench.recorded_traffic("w", "eager", "l2_write_bytes_per_launch") == 7.0
     assert bench.recorded_traffic("w", "merge") is None
+
+
+def test_expected_live_lengths_follow_the_steps_taken():
+    wl = synth.GLA_DIAG
+    R = 6
+    go = bench.phase_offsets(wl, R, "spread")
+    for n in (0, 1, 5, 6, 7, 53):
+        want = bench.expected_live_lengths(wl, go, n)
+        for g in range(R):
+            taken = len([j for j in range(n) if j % R == g])
+            np.testing.assert_array_equal(want[g], (go[g] + taken) % wl.log_cap)
+    assert not bench.expected_live_lengths(wl, go, 9, merge_every=True).any()

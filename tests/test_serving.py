@@ -106,10 +106,11 @@ def _prefill(r):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("tile_v,log_format,log_cap", [(0, "fp32", LOG_CAP), (128, "fp32", LOG_CAP),
-                                                      (0, "compact", LOG_CAP), (128, "compact", LOG_CAP),
-                                                      (0, "fp32", "auto"), (128, "compact", "auto")])
-def test_server_requests_match_the_oracle(tile_v, log_format, log_cap):
+@pytest.mark.parametrize("tile_v,log_format,log_cap,merge", [
+    (0, "fp32", LOG_CAP, "capacity"), (128, "fp32", LOG_CAP, "capacity"),
+    (0, "compact", LOG_CAP, "capacity"), (128, "compact", LOG_CAP, "capacity"),
+    (0, "fp32", "auto", "capacity"), (128, "compact", "auto", "capacity"), (0, "fp32", LOG_CAP, "adaptive")])
+def test_server_requests_match_the_oracle(tile_v, log_format, log_cap, merge):
     import torch
     from oracle import eager_tasks
     from recurrent_state_serving_b200 import tuning
@@ -117,7 +118,7 @@ def test_server_requests_match_the_oracle(tile_v, log_format, log_cap):
     from tests import harness as Hn
     srv = DecodeServer(n_slots=6, n_layers=L_LAYERS, n_heads=H, n_kheads=HK, d_k=D, d_v=D,
                        log_cap=log_cap, decay="diag", update="delta", log_format=log_format,
-                       tile_v=tile_v, max_batch=5)
+                       tile_v=tile_v, max_batch=5, merge=merge)
     if log_cap == "auto":
         # the modelled interval of this operator, which the schedule's requests outlive
         assert srv.log_cap == tuning.auto_log_cap(D, D, "diag", "delta", log_format)
