@@ -208,11 +208,12 @@ def group_live_entries(group_offsets, step_index: int, log_cap: int):
 
 def expected_live_lengths(wl, group_offsets, n_steps: int, merge_every: bool = False):
     """Live entries of every slot of every group ([n_groups, batch]) after global steps
-    0 .. n_steps-1 (step j on group j mod R), as the byte accounting assumes."""
+    0 .. n_steps-1 (step j on group j mod R), as the byte accounting assumes.  Merging
+    every step, a group keeps its pre-step live lengths until its first step."""
     R = group_offsets.shape[0]
     taken = np.array([(n_steps - g + R - 1) // R for g in range(R)])
     if merge_every:
-        return np.zeros_like(group_offsets)
+        return np.where(taken[:, None] > 0, 0, group_offsets)
     return (group_offsets + taken[:, None]) % wl.log_cap
 
 
@@ -227,8 +228,13 @@ def timed_window_bytes(wl, group_offsets, first: int, K: int, log_format: str = 
     scale = wl.n_heads * wl.n_layers
     hist = np.zeros(L, np.int64)
     if merge_every:
-        hist[0] = K * wl.batch
-        return hist[0] * traffic.deferred_head_step(wl, 0, merge=True, log_format=log_format) * scale, hist
+        # a group's first step folds its pre-step entries; every later step starts empty
+        R = group_offsets.shape[0]
+        for j in range(first, first + K):
+            c = group_offsets[j % R] if j // R == 0 else np.zeros(wl.batch, np.int64)
+            hist += np.bincount(c, minlength=L)
+        per_c = [traffic.deferred_head_step(wl, c, merge=True, log_format=log_format) for c in range(L)]
+        return float(np.dot(hist, per_c)) * scale, hist
     per_c = [traffic.deferred_head_step(wl, c, merge=(c == L - 1), log_format=log_format) for c in range(L)]
     for j in range(first, first + K):
         hist += np.bincount(group_live_entries(group_offsets, j, L), minlength=L)

@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
         } else {
             const int y = x - hd.nl + (hd.part ? (hd.part - 1) * (NCH / hd.np) : 0);  // a part's first chunk
-            const bool keep = y < NCH && (hd.mk == MK_PASS2 || hd.mk == MK_ROUNDS);
+            const bool keep = y < NCH && hd.mk == MK_ROUNDS;
             ptx::mbar_arrive_expect_tx(bar, CB);
             ptx::bulk_g2s(dst, p.state + hd.head * (size_t)(DK * DV) + (size_t)(y & (NCH - 1)) * CF, CB, bar,
                           keep ? pol_keep : pol_stream);
@@ -738,7 +738,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             // shared memory: e^{lbar_t} Sbar + sum_i A'_i b_i^T + k b_t^T, i ascending.
             // A'_i rows of the block are published AG entries at a time by the block's
             // four owner lanes and read by every lane as broadcasts.
-            auto write_rows = [&](const float *sb, int cx, const float4 &bt4) {
+            // (token: add k b_t^T; streaming: evict-first stores, else plain stores that
+            //  stay in L2 for pass 2 of a delta-rule merge)
+            auto write_rows = [&](const float *sb, int cx, const float4 &bt4, bool token, bool streaming) {
                 float4 acc[CR];
 #pragma unroll
                 for (int r4 = 0; r4 < CR / 4; ++r4) {
@@ -784,8 +786,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
                         const int rr = 4 * r4 + y;
-                        fma4(acc[rr], kv[y], bt4);
-                        __stcs(reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane, acc[rr]);
+                        if (token) fma4(acc[rr], kv[y], bt4);
+                        float4 *dst = reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane;
+                        if (streaming) __stcs(dst, acc[rr]);
+                        else *dst = acc[rr];
                     }
                 }
             };
@@ -814,7 +818,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                         if (DELTA) fma4(Yk, kv[y], S);
                     }
                 }
-                if (!DELTA && mk == MK_FUSED) write_rows(sb, cx, v4);
+                if (!DELTA && mk == MK_FUSED) {
+                    write_rows(sb, cx, v4, true, true);
+                } else if (DELTA && mk == MK_PASS2) {
+                    // e^{lbar_t} Sbar + sum_i A'_i b_i^T now, while the stream is DRAM-bound;
+                    // the token term needs b_t, so pass 2 adds it.  Pass 2's bulk copies
+                    // re-read these rows (issued at least NCH - NSW stages later): order
+                    // the writes before them.
+                    write_rows(sb, cx, v4, false, false);
+                    ptx::fence_proxy_async_global();
+                }
                 release();
             }
             if (abort) break;
@@ -868,10 +881,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
                     *reinterpret_cast<float4 *>(ent + LO + 4 * lane) = reinterpret_cast<const float4 *>(rv_l)[lane];
                 if (DECAY == DL_DECAY_SCALAR && lane == 0) ent[LO] = rv_l[0];
             } else if (mk == MK_PASS2) {
-                // -- pass 2: the tile again (from L2), rewritten row block by row block
+                // -- pass 2: the rows pass 1 wrote, again (from L2), plus the token term
+                //    k b_t^T, row block by row block
                 for (int cx = 0; cx < NCH; ++cx) {
                     if (!wait_chunk()) { abort = true; break; }
-                    write_rows(st + (size_t)(gc % NSW) * CF, cx, bt4);
+                    const float *sb = st + (size_t)(gc % NSW) * CF;
+#pragma unroll
+                    for (int r4 = 0; r4 < CR / 4; ++r4) {
+                        const float4 k4 = reinterpret_cast<const float4 *>(rv_k + cx * CR)[r4];
+                        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) {
+                            const int rr = 4 * r4 + y;
+                            float4 S = reinterpret_cast<const float4 *>(sb + rr * DV)[lane];
+                            fma4(S, kv[y], bt4);
+                            __stcs(reinterpret_cast<float4 *>(tile + (size_t)(cx * CR + rr) * DV) + lane, S);
+                        }
+                    }
                     release();
                 }
                 if (abort) break;

@@ -248,4 +248,23 @@ def test_expected_live_lengths_follow_the_steps_taken():
         for g in range(R):
             taken = len([j for j in range(n) if j % R == g])
             np.testing.assert_array_equal(want[g], (go[g] + taken) % wl.log_cap)
-    assert not bench.expected_live_lengths(wl, go, 9, merge_every=True).any()
+    # merging every step: stepped groups are empty, the others keep their offsets
+    ev = bench.expected_live_lengths(wl, go, 4, merge_every=True)
+    assert not ev[:4].any()
+    np.testing.assert_array_equal(ev[4:], go[4:])
+
+
+def test_merge_every_window_counts_each_groups_first_fold():
+    """Under the adaptive policy a group's first step folds its pre-step entries (a
+    merge with c > 0); its later steps start empty."""
+    wl = synth.GDN_GVA
+    R = bench.rotation_groups(wl, "rotate")
+    go = bench.phase_offsets(wl, R, "spread")
+    L = wl.log_cap
+    b, hist = bench.timed_window_bytes(wl, go, 3, 10, merge_every=True)
+    want = np.bincount(go[3:13, 0], minlength=L)
+    np.testing.assert_array_equal(hist, want)
+    per_c = [traffic.deferred_head_step(wl, c, merge=True) for c in range(L)]
+    assert b == pytest.approx(float(np.dot(want, per_c)) * wl.n_heads * wl.n_layers)
+    _, hist2 = bench.timed_window_bytes(wl, go, R, 5, merge_every=True)   # second round: empty
+    assert hist2[0] == 5 and hist2[1:].sum() == 0
