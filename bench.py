@@ -1006,7 +1006,14 @@ def run_gpu(a, wl, rank, world, dist):
     subs = []
     for swl in spec_list(a.subs):
         Ks = sub_steps(swl, K, a.log_format)
-        srec, _ = measure_decode(ctx, swl, Ks, max(W, 3))
+        Ws = max(W, 3)
+        from recurrent_state_serving_b200 import deltalog as dl
+        if dl.dl_merge_policy(swl.batch, swl.n_heads, a.merge):
+            # merging every step: a group's first step folds the log its staggering
+            # pre-steps left; warm up one whole rotation so that the window is the
+            # steady state (every slot starting empty)
+            Ws = max(Ws, rotation_groups(swl, a.l2))
+        srec, _ = measure_decode(ctx, swl, Ks, Ws)
         subs.append(srec)
     if subs:
         result["subs"] = subs

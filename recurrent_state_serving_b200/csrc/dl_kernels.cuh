@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include "dl_internal.h"
+#include "dl_ptx.cuh"
 
 namespace dl {
 
@@ -572,21 +573,27 @@ __global__ void __launch_bounds__(MH_NT, 2) merge_head_kernel(const KParams p, c
     for (int r = 0; r < RW; ++r)
         S[r] = __ldcs(reinterpret_cast<const float4 *>(tile + (size_t)(RW * w + r) * D) + lane);
 
-    // 2. lbar = Lambda_{c-1}, e^{lbar}; A'^T and b of the live entries
+    // 2. the live entries, copied raw into shared memory with per-thread asynchronous
+    //    16-byte copies as soon as c is known (lbar = Lambda_{c-1} arrives with them);
+    //    then e^{lbar}, A'^T and b from shared memory
     const float *ring = p.log + head * (size_t)p.L * p.E;
     float *sA = s_dyn;                        // [c][D]  A'^T
     float *sB = s_dyn + (size_t)p.L * D;      // [c][D]  b
+    float *sRaw = s_dyn + (size_t)2 * p.L * D;  // [c][E]  the entries as stored
+    for (int idx = tid; idx < c * p.E / 4; idx += MH_NT) ptx::cp_async16(sRaw + 4 * idx, ring + 4 * idx);
+    ptx::cp_async_wait_all();
+    __syncthreads();
     for (int r = tid; r < D; r += MH_NT) {
         float lb = 0.f;
-        if (c > 0 && DECAY == DL_DECAY_DIAG) lb = ring[(size_t)(c - 1) * p.E + p.loff + r];
-        if (c > 0 && DECAY == DL_DECAY_SCALAR) lb = ring[(size_t)(c - 1) * p.E + p.loff];
+        if (c > 0 && DECAY == DL_DECAY_DIAG) lb = sRaw[(size_t)(c - 1) * p.E + p.loff + r];
+        if (c > 0 && DECAY == DL_DECAY_SCALAR) lb = sRaw[(size_t)(c - 1) * p.E + p.loff];
         s_lb[r] = lb;
         s_e[r] = DECAY == DL_DECAY_NONE ? 1.f : expf(lb);
     }
     __syncthreads();
     for (int idx = tid; idx < c * (D / 4); idx += MH_NT) {
         const int i = idx / (D / 4), r4 = idx % (D / 4);
-        const float *ent = ring + (size_t)i * p.E;
+        const float *ent = sRaw + (size_t)i * p.E;
         float4 a4 = ent_a4(p, ent, r4);
         if (DECAY == DL_DECAY_DIAG) {
             const float4 L4 = *reinterpret_cast<const float4 *>(ent + p.loff + 4 * r4);

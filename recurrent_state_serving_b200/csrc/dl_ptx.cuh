@@ -71,6 +71,16 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Per-thread asynchronous 16-byte copy global -> shared (both 16-byte aligned),
+// cached in L2 only; cp_async_wait_all waits for all of the thread's copies.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // L2 policy: keep the line (data read again soon).
 __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t pol;

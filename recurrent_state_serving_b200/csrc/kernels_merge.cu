@@ -73,12 +73,13 @@ namespace {
 
 template <int DECAY>
 cudaError_t merge_head_one(const KParams &p, bool materialize, cudaStream_t st) {
-    const size_t smem = (size_t)2 * p.L * 128 * sizeof(float);
+    // A'^T and b (2 x L x 128 floats) and the raw entries (L x E floats)
+    const size_t smem = ((size_t)2 * p.L * 128 + (size_t)p.L * p.E) * sizeof(float);
     auto kern = merge_head_kernel<DECAY>;
-    static bool configured = false;  // per instantiation: room for the largest log (64 entries)
+    static bool configured = false;  // per instantiation: room for the largest log (64 fp32 entries)
     if (!configured) {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   2 * 64 * 128 * (int)sizeof(float));
+                                                   (2 * 64 * 128 + 64 * 384) * (int)sizeof(float));
         if (e != cudaSuccess) return e;
         configured = true;
     }
