@@ -580,7 +580,14 @@ __global__ void __launch_bounds__(MH_NT, 2) merge_head_kernel(const KParams p, c
     float *sA = s_dyn;                        // [c][D]  A'^T
     float *sB = s_dyn + (size_t)p.L * D;      // [c][D]  b
     float *sRaw = s_dyn + (size_t)2 * p.L * D;  // [c][E]  the entries as stored
-    for (int idx = tid; idx < c * p.E / 4; idx += MH_NT) ptx::cp_async16(sRaw + 4 * idx, ring + 4 * idx);
+    // the part of a row the merge reads: whole rows when they hold nothing unused
+    // (per-key decay, compact rows), else a | b | Lambda_0 (scalar decay) or a | b
+    const int ecopy = (p.a16 || DECAY == DL_DECAY_DIAG) ? p.E : DECAY == DL_DECAY_SCALAR ? p.loff + 4 : p.loff;
+    const int nv = ecopy / 4;  // 16-byte vectors per entry
+    for (int idx = tid; idx < c * nv; idx += MH_NT) {
+        const size_t o = (size_t)(idx / nv) * p.E + 4 * (idx % nv);
+        ptx::cp_async16(sRaw + o, ring + o);
+    }
     ptx::cp_async_wait_all();
     __syncthreads();
     for (int r = tid; r < D; r += MH_NT) {

@@ -100,10 +100,11 @@ constexpr int NPA = 8;                      // split heads in flight per CTA (ac
 // balanced schedule: the whole batch's slot ids and live lengths, and a bitmap of its
 // merging rows with per-word prefix counts
 constexpr int BAL_ROWS = 512;
+constexpr int LMAX = 64;                    // largest log capacity (bins of the longest-first order)
 constexpr int BAL_WORDS = BAL_ROWS / 32;
 constexpr size_t SMEM = (size_t)NW * NSW * CB + (size_t)NW * WSCR * 4 + (size_t)NW * NB * 8 + 32 +
                         (size_t)KMAX * (4 + 4 + 4 + 4) + (size_t)2 * KMAX * 2 + (size_t)NPA * DV * 4 +
-                        (size_t)BAL_ROWS * (4 + 1) + (size_t)BAL_WORDS * (4 + 4);
+                        (size_t)BAL_ROWS * (4 + 1) + (size_t)BAL_WORDS * (4 + 4) + (size_t)(LMAX + 2) * 4;
 static_assert(KMAX + (MAX_PARTS - 1) * NPA <= 2 * KMAX, "the order holds every head and every extra part");
 static_assert(SMEM <= 232448, "a CTA may use at most 227 KB of shared memory");
 static_assert(NSW == 3, "the round-wise merge uses stages 0-1 for the tile and stage 2 as scratch");
@@ -227,7 +228,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     int *row_slot = reinterpret_cast<int *>(pacc + NPA * DV);   // balanced schedule: per batch row
     unsigned *bmap = reinterpret_cast<unsigned *>(row_slot + BAL_ROWS);  // merging rows
     int *wpre = reinterpret_cast<int *>(bmap + BAL_WORDS);      // set bits before each word
-    uint8_t *row_len = reinterpret_cast<uint8_t *>(wpre + BAL_WORDS);
+    // append heads per live length, then the next position of each (longest first)
+    int *lbin = wpre + BAL_WORDS;
+    uint8_t *row_len = reinterpret_cast<uint8_t *>(lbin + LMAX + 2);
 
     // merges with live entries need tensor memory (auto-merge decode steps only)
     const bool use_tm = p.auto_merge && !p.eager && p.log != nullptr;
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
     }
     for (int i = threadIdx.x; i < NPA * DV; i += NTHREADS) pacc[i] = 0.f;
     for (int i = threadIdx.x; i < BAL_WORDS; i += NTHREADS) bmap[i] = 0u;
+    for (int i = threadIdx.x; i < LMAX + 2; i += NTHREADS) lbin[i] = 0;
     if (use_tm && w == 0) {
         ptx::tmem_alloc(tm_slot, TM_COLS);
         ptx::tmem_relinquish();
@@ -387,7 +391,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             }
             comb[k] = cm;
             if (merges(s, c)) atomicAdd(&cnt[0], np);
+            else atomicAdd(&lbin[c < 0 || c > LMAX ? 0 : c], 1);
             if (np > 1) atomicAdd(&cnt[3], np - 1);
+        }
+        __syncthreads();
+        // Append heads in order of decreasing live length (longest first): a head with
+        // c live entries streams and replays c log entries besides its tile, so the
+        // short ones end the order and the warps finish closer together.  lbin[c]
+        // becomes the first append position of live length c.
+        if (threadIdx.x == 0) {
+            int acc = 0;
+            for (int cc = LMAX; cc >= 0; --cc) {
+                const int n = lbin[cc];
+                lbin[cc] = acc;
+                acc += n;
+            }
         }
         __syncthreads();
         const int nm = cnt[0];
@@ -411,7 +429,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) warp_head_kernel(const KParams p)
             } else if (merges(s, c)) {
                 order[merge_pos(atomicAdd(&cnt[1], 1))] = (uint16_t)k;
             } else {
-                const int a = atomicAdd(&cnt[2], 1);
+                const int a = atomicAdd(&lbin[c < 0 || c > LMAX ? 0 : c], 1);  // longest first
                 int pos = a;  // the a-th position no merge head takes
                 if (spread) {
                     for (int i = 0; i < nm && merge_pos(i) <= pos; ++i) ++pos;
