@@ -110,8 +110,9 @@ struct DynLayout {
 // then either append (k, b_t, lbar_t) as entry c, or, on the slot's merge step
 // (on every step with p.merge_every, and always in eager mode), write
 //   S_t = e^{lbar_t} (.) Sbar + sum_i A'_i b_i^T + k b_t^T,  A'_i = a_i (.) e^{lbar_t - Lambda_i}.
+// ME: the instantiation for launches that merge every step (p.merge_every).
 // ---------------------------------------------------------------------------
-template <int DK, int BV, int DECAY, bool DELTA, typename IT>
+template <int DK, int BV, int DECAY, bool DELTA, typename IT, bool ME = false>
 __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     step_kernel(const KParams p)
 {
@@ -182,6 +183,13 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     float *ring = p.log ? p.log + head * (size_t)p.L * p.E : nullptr;
     const DynLayout lay(p.L, BV);
     float *s_cq = s_dyn + lay.cq, *s_ck = s_dyn + lay.ck, *s_b = s_dyn + lay.b, *s_A = s_dyn + lay.A;
+    // A merge stages the A'_i rows in shared memory, except in launches that merge
+    // every step (their own instantiation, so that the others keep their registers):
+    // those are sized like an eager step, without the A' area (on B200 the larger
+    // allocation cost about 0.4 us per 32-head launch), and the rare merge of a
+    // non-empty log there (the first step after the policy changes) forms A'_i in the
+    // update loop instead, with the same arithmetic.
+    constexpr bool stage_A = !ME;
 
     // 3. token, cumulative log-decay, prescaled q and k
     const int g = h / (p.H / p.Hk);
@@ -261,7 +269,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
                     }
                     pq = fmaf(w, s_q[r], pq);
                     if (DELTA) pk = fmaf(wk, s_k[r], pk);
-                    if (merge_now) s_A[i * DK + r] = w;
+                    if (stage_A && merge_now) s_A[i * DK + r] = w;
                 }
             }
             pqv[u] = pq;
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
                 if (DELTA) s_ck[i] = *cluster.map_shared_rank(s_ck + i, o);
             }
         }
-        if (merge_now) {
+        if (stage_A && merge_now) {
             for (int idx = tid; idx < c * DK; idx += NT) {
                 const int o = (idx / DK / NW) % cl;
                 if (o != cr) s_A[idx] = *cluster.map_shared_rank(s_A + idx, o);
@@ -398,8 +406,19 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         }
         for (int i = 0; i < c; ++i) {
             const float4 b4 = reinterpret_cast<const float4 *>(s_b + i * BV)[quad];
+            if constexpr (stage_A) {
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) fma4(Sr[m], s_A[i * DK + rg + m * RG], b4);
+                for (int m = 0; m < RPT; ++m) fma4(Sr[m], s_A[i * DK + rg + m * RG], b4);
+            } else {
+                const float *ent = ring + (size_t)i * p.E;
+                const float fs = DECAY == DL_DECAY_SCALAR ? expf(s_ell[0] - ent[p.loff]) : 1.f;
+#pragma unroll
+                for (int m = 0; m < RPT; ++m) {
+                    const int r = rg + m * RG;
+                    const float a = ent_a(p, ent, r);
+                    fma4(Sr[m], DECAY == DL_DECAY_DIAG ? a * expf(s_ell[r] - ent[p.loff + r]) : a * fs, b4);
+                }
+            }
         }
 #pragma unroll
         for (int m = 0; m < RPT; ++m)

@@ -494,6 +494,23 @@ def test_split_merge_heads_match_the_oracle(shape, staggered, log_format):
     H.check_steps(states[0], se[0], tol=H.REL_L2_GPU, elem=None, what="state")
 
 
+@pytest.mark.parametrize("batch", [64, 128])
+def test_split_heads_are_the_same_on_every_run(batch):
+    """Two runs of the same staggered workload agree bit for bit (outputs, logs, live
+    lengths, states): at seven heads per CTA (no head list) and at about fourteen
+    (balanced schedule, merge heads split in two halves whose sum does not depend on
+    which half ends first), whatever order the warps take their heads in."""
+    wl = synth.GLA_DIAG.with_(batch=batch, n_heads=16, n_kheads=16, steps=20, log_cap=8, staggered=True)
+    res = []
+    for _ in range(2):
+        r = DecodeRunner(wl, tile_v=128)
+        o, _, _ = H.gpu_rollout(r, wl.steps)
+        assert r.errors() == 0
+        res.append((torch.as_tensor(o[0]), r.pool.log.clone(), r.pool.log_len.clone(), r.pool.state.clone()))
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)
+
+
 def test_expired_wait_sets_the_timeout_bit_and_the_pool_recovers():
     """A wait of the whole-head kernel made to run out (test hook: one warp waits, for
     at most 2 ms, on a barrier nothing completes, with its first bulk copies in
