@@ -110,9 +110,8 @@ struct DynLayout {
 // then either append (k, b_t, lbar_t) as entry c, or, on the slot's merge step
 // (on every step with p.merge_every, and always in eager mode), write
 //   S_t = e^{lbar_t} (.) Sbar + sum_i A'_i b_i^T + k b_t^T,  A'_i = a_i (.) e^{lbar_t - Lambda_i}.
-// ME: the instantiation for launches that merge every step (p.merge_every).
 // ---------------------------------------------------------------------------
-template <int DK, int BV, int DECAY, bool DELTA, typename IT, bool ME = false>
+template <int DK, int BV, int DECAY, bool DELTA, typename IT>
 __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     step_kernel(const KParams p)
 {
@@ -184,12 +183,15 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
     const DynLayout lay(p.L, BV);
     float *s_cq = s_dyn + lay.cq, *s_ck = s_dyn + lay.ck, *s_b = s_dyn + lay.b, *s_A = s_dyn + lay.A;
     // A merge stages the A'_i rows in shared memory, except in launches that merge
-    // every step (their own instantiation, so that the others keep their registers):
-    // those are sized like an eager step, without the A' area (on B200 the larger
-    // allocation cost about 0.4 us per 32-head launch), and the rare merge of a
-    // non-empty log there (the first step after the policy changes) forms A'_i in the
-    // update loop instead, with the same arithmetic.
-    constexpr bool stage_A = !ME;
+    // every step with scalar decay (RetNet, GDN): those are sized like an eager step,
+    // without the A' area (on B200 the larger allocation cost about 0.4 us per
+    // 32-head launch), and the rare merge of a non-empty log there (the first step
+    // after the policy changes) forms A'_i in the update loop instead, with the same
+    // arithmetic.  For the other decays that loop changed the registers of every
+    // launch of the instantiation (per-key decay: the eager GLA B = 64 step went from
+    // 26 to 33 us), so they keep the staged rows.
+    constexpr bool RECOMPUTE_OK = DECAY == DL_DECAY_SCALAR;
+    const bool stage_A = !(RECOMPUTE_OK && p.merge_every);
 
     // 3. token, cumulative log-decay, prescaled q and k
     const int g = h / (p.H / p.Hk);
@@ -406,18 +408,14 @@ __global__ void __launch_bounds__(TileShape<DK, BV>::NT)
         }
         for (int i = 0; i < c; ++i) {
             const float4 b4 = reinterpret_cast<const float4 *>(s_b + i * BV)[quad];
-            if constexpr (stage_A) {
+            if (!RECOMPUTE_OK || stage_A) {
 #pragma unroll
                 for (int m = 0; m < RPT; ++m) fma4(Sr[m], s_A[i * DK + rg + m * RG], b4);
-            } else {
+            } else if constexpr (RECOMPUTE_OK) {
                 const float *ent = ring + (size_t)i * p.E;
-                const float fs = DECAY == DL_DECAY_SCALAR ? expf(s_ell[0] - ent[p.loff]) : 1.f;
+                const float fs = expf(s_ell[0] - ent[p.loff]);
 #pragma unroll
-                for (int m = 0; m < RPT; ++m) {
-                    const int r = rg + m * RG;
-                    const float a = ent_a(p, ent, r);
-                    fma4(Sr[m], DECAY == DL_DECAY_DIAG ? a * expf(s_ell[r] - ent[p.loff + r]) : a * fs, b4);
-                }
+                for (int m = 0; m < RPT; ++m) fma4(Sr[m], ent_a(p, ent, rg + m * RG) * fs, b4);
             }
         }
 #pragma unroll

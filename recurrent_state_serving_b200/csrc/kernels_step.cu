@@ -14,11 +14,11 @@ namespace {
 template <int BV, int DECAY, bool DELTA, typename IT>
 cudaError_t launch_one(const KParams &p, cudaStream_t st) {
     using Sh = TileShape<DL_STEP_DK, BV>;
-    // merge-every launches form A' without shared memory (step_kernel)
-    const size_t smem = dyn_floats(p.L, DL_STEP_DK, BV, p.auto_merge != 0 && !p.merge_every) * sizeof(float);
+    // merge-every launches with scalar decay form A' without shared memory (step_kernel)
+    const bool need_A = p.auto_merge != 0 && !(p.merge_every && DECAY == DL_DECAY_SCALAR);
+    const size_t smem = dyn_floats(p.L, DL_STEP_DK, BV, need_A) * sizeof(float);
     const long long grid = (long long)p.batch * p.H * p.nv;
-    auto kern = p.merge_every ? step_kernel<DL_STEP_DK, BV, DECAY, DELTA, IT, true>
-                              : step_kernel<DL_STEP_DK, BV, DECAY, DELTA, IT, false>;
+    auto kern = step_kernel<DL_STEP_DK, BV, DECAY, DELTA, IT>;
     if (p.cl <= 1) {
         kern<<<(unsigned)grid, Sh::NT, smem, st>>>(p);
         return cudaGetLastError();
