@@ -91,6 +91,33 @@ int main(void) {
     expect(dl_decode_step(pool, 0, &a, 1, NULL) == DL_ERR_SHAPE, "oversized batch");
     expect(dl_read_error(pool, NULL, 0, NULL) == DL_ERR_INVALID_ARG, "read_error without output");
     expect(dl_destroy_pool(pool) == DL_OK, "dl_destroy_pool");
+
+    /* the allocation-free step: host checks only (batch 0 returns before any CUDA call) */
+    a.batch = 0;
+    expect(dl_decode_step_noalloc(&d, 0, &a, DL_MERGE_ADAPTIVE, NULL) == DL_OK, "noalloc empty step");
+    expect(dl_decode_step_noalloc(NULL, 0, &a, DL_MERGE_ADAPTIVE, NULL) == DL_ERR_INVALID_ARG,
+           "noalloc without descriptor");
+    expect(dl_decode_step_noalloc(&d, 2, &a, DL_MERGE_ADAPTIVE, NULL) == DL_ERR_INVALID_ARG,
+           "noalloc layer out of range");
+    {
+        dl_pool_desc big = d;
+        big.n_slots = DL_NOALLOC_MAX_COUNTERS; /* x 2 layers: more counters than the array */
+        expect(dl_decode_step_noalloc(&big, 0, &a, DL_MERGE_ADAPTIVE, NULL) == DL_ERR_SHAPE,
+               "noalloc counter limit");
+    }
+
+    /* merge policy: at capacity never merges every step; adaptive does below a few
+       heads per SM (one 32-head slot) and does not for a launch that fills the GPU */
+    int32_t every = -1;
+    expect(dl_merge_policy(1, 32, DL_MERGE_ADAPTIVE, NULL) == DL_ERR_INVALID_ARG, "merge_policy without output");
+    expect(dl_merge_policy(-1, 32, DL_MERGE_ADAPTIVE, &every) == DL_ERR_INVALID_ARG, "merge_policy negative batch");
+    expect(dl_merge_policy(1, 32, DL_MERGE_AT_CAPACITY, &every) == DL_OK && every == 0, "capacity policy");
+    expect(dl_merge_policy(1, 32, DL_MERGE_ADAPTIVE, &every) == DL_OK && every == 1, "adaptive, one slot");
+    expect(dl_merge_policy(256, 32, DL_MERGE_ADAPTIVE, &every) == DL_OK && every == 0, "adaptive, full launch");
+    printf("merge_policy ok\n");
+
+    /* the stall test hook is host state only; 0 switches it off */
+    expect(dl_debug_stall(0) == DL_OK, "dl_debug_stall off");
     expect(dl_status_string(DL_OK) != NULL && dl_status_string(DL_ERR_SHAPE) != NULL, "status strings");
 
     d.d_k = 0;
