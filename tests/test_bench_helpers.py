@@ -268,3 +268,26 @@ def test_merge_every_window_counts_each_groups_first_fold():
     assert b == pytest.approx(float(np.dot(want, per_c)) * wl.n_heads * wl.n_layers)
     _, hist2 = bench.timed_window_bytes(wl, go, R, 5, merge_every=True)   # second round: empty
     assert hist2[0] == 5 and hist2[1:].sum() == 0
+
+
+def test_reference_arm_prints_the_oracle_line():
+    """bench.py --impl reference times the fp64 oracle on the host cores (no GPU) and
+    prints one JSON line with the same metric, unit and config as the GPU arm."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    run = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", "gla_rwkv6_diag:b4", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert run.returncode == 0, run.stderr[-2000:]
+    lines = [ln for ln in run.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["dtype"] == "f64"
+    assert d["config"]["workload"] == "gla_rwkv6_diag_b4_h16_d128_L8"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
