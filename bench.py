@@ -1122,7 +1122,8 @@ def main(argv=None):
     wl = workload(a)
     if a.traffic_from:
         kern = {"decode": r"warp_head_kernel|step_kernel", "eager": r"step_kernel",
-                "merge": r"merge_kernel", "materialize": r"merge_kernel"}[a.traffic_kind]
+                "merge": r"merge_kernel|merge_head_kernel",
+                "materialize": r"merge_kernel|merge_head_kernel"}[a.traffic_kind]
         text = traffic_summary_from_ncu(a.traffic_from, workload_key(wl, a.log_format), kern, a.traffic_kind)
         with open(PROFILE_TRAFFIC, "a") as f:
             f.write(text + "\n")

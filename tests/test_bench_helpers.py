@@ -291,3 +291,18 @@ def test_reference_arm_prints_the_oracle_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun the reference arm runs and prints on rank 0 alone; any other rank
+    exits 0 without work or output."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    run = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", "gla_rwkv6_diag:b4", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root, env=env)
+    assert run.returncode == 0, run.stderr[-2000:]
+    assert not [ln for ln in run.stdout.splitlines() if ln.startswith("{")]
